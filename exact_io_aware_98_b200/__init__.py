@@ -1,0 +1,196 @@
+"""Python binding of libfa (exact IO-aware attention on B200, sm_100a).
+
+Argument marshalling only: every step of the attention computation runs in the
+CUDA kernels behind the C ABI declared in ``include/fa.h``.  PyTorch supplies
+device memory and the current stream.  There is no CPU fallback: if the
+library is missing or no GPU is present, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_BF16, FA_F32 = 0, 1
+_STATUS = {0: "FA_OK", -1: "FA_ERR_INVALID", -2: "FA_ERR_UNSUPPORTED", -3: "FA_ERR_ALIGN",
+           -4: "FA_ERR_CUDA", -5: "FA_ERR_TIMEOUT", -6: "FA_ERR_WORKSPACE"}
+
+# exported symbol -> (restype, argtypes)
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "fa_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp, _i, _vp]),
+    "fa_bwd_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "fa_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp,
+                    _vp, _i, _vp, _sz, _vp]),
+    "fa_fwd_tile_reference": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp,
+                                   _i, _vp]),
+    "fa_naive_workspace_size": (_sz, [_i, _i, _i]),
+    "fa_naive_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz,
+                          _vp]),
+    "fa_get_last_error": (ctypes.c_char_p, []),
+    "fa_device_status": (_i, [ctypes.POINTER(ctypes.c_uint)]),
+}
+
+_lib = None
+
+
+class FaError(RuntimeError):
+    pass
+
+
+def load(path: str = LIB_PATH):
+    """Load libfa.so (built by ``exact_io_aware_98_b200.build``); raises if absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise FaError(f"libfa.so not found at {path}: build it first "
+                          "(python -m exact_io_aware_98_b200.build)")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        msg = load().fa_get_last_error().decode(errors="replace")
+        raise FaError(f"{what}: {_STATUS.get(rc, rc)}: {msg}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _require(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise FaError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise FaError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise FaError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _masks(block_mask, kv_len):
+    if block_mask is not None:
+        _require(block_mask, "block_mask", torch.uint8)
+    if kv_len is not None:
+        _require(kv_len, "kv_len", torch.int32)
+    return _ptr(block_mask), _ptr(kv_len)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    if t.dtype == torch.float32:
+        return FA_F32
+    raise FaError(f"unsupported dtype {t.dtype}")
+
+
+def default_scale(d: int) -> float:
+    return float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32).item())
+
+
+def fwd(q, k, v, scale: Optional[float] = None, causal: bool = False, block_mask=None,
+        kv_len=None, out=None, lse=None):
+    """O, lse = fa_fwd(q, k, v); tensors [B, H, N, d] (bf16 or fp32) on the GPU."""
+    lib = load()
+    B, H, N, d = q.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _require(t, n, q.dtype)
+        if t.shape != q.shape:
+            raise FaError(f"{n} shape {tuple(t.shape)} != q shape {tuple(q.shape)}")
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _require(o, "out", q.dtype)
+    _require(l, "lse", torch.float32)
+    bm, kl = _masks(block_mask, kv_len)
+    s = default_scale(d) if scale is None else float(scale)
+    rc = lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, H, N, d, s, int(causal),
+                    bm, kl, _dtype_code(q), _stream())
+    _check(rc, "fa_fwd")
+    return o, l
+
+
+def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(load().fa_bwd_workspace_size(B, H, N, d))
+
+
+def bwd(q, k, v, o, lse, do, scale: Optional[float] = None, causal: bool = False,
+        block_mask=None, kv_len=None, workspace=None, dq=None, dk=None, dv=None):
+    """dQ, dK, dV = fa_bwd(...); bf16 tensors [B, H, N, d] on the GPU."""
+    lib = load()
+    B, H, N, d = q.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _require(t, n, q.dtype)
+    _require(lse, "lse", torch.float32)
+    need = bwd_workspace_size(B, H, N, d)
+    ws = torch.empty(need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    _require(ws, "workspace", torch.uint8)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    bm, kl = _masks(block_mask, kv_len)
+    s = default_scale(d) if scale is None else float(scale)
+    rc = lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                    _ptr(dv), B, H, N, d, s, int(causal), bm, kl, _dtype_code(q), _ptr(ws),
+                    ws.numel(), _stream())
+    _check(rc, "fa_bwd")
+    return dq, dk, dv
+
+
+def fwd_tile_reference(q, k, v, bc: int, scale: Optional[float] = None, causal: bool = False,
+                       block_mask=None, kv_len=None):
+    """bf16 CUDA-core forward that rescales after every `bc` keys (deviation study)."""
+    lib = load()
+    B, H, N, d = q.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _require(t, n, torch.bfloat16)
+    o = torch.empty_like(q)
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    bm, kl = _masks(block_mask, kv_len)
+    s = default_scale(d) if scale is None else float(scale)
+    rc = lib.fa_fwd_tile_reference(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, H, N, d, s,
+                                   int(causal), bm, kl, int(bc), _stream())
+    _check(rc, "fa_fwd_tile_reference")
+    return o, l
+
+
+def naive_fwd(q, k, v, scale: Optional[float] = None, causal: bool = False, block_mask=None,
+              kv_len=None, workspace=None):
+    """Materialised baseline: S and P go through HBM in bf16."""
+    lib = load()
+    B, H, N, d = q.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _require(t, n, torch.bfloat16)
+    need = int(lib.fa_naive_workspace_size(B, H, N))
+    ws = torch.empty(need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    o = torch.empty_like(q)
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    bm, kl = _masks(block_mask, kv_len)
+    s = default_scale(d) if scale is None else float(scale)
+    rc = lib.fa_naive_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, H, N, d, s,
+                          int(causal), bm, kl, _ptr(ws), ws.numel(), _stream())
+    _check(rc, "fa_naive_fwd")
+    return o, l
+
+
+def device_status() -> int:
+    """Synchronise; return the bounded-wait status code (0 = no wait gave up) and clear it."""
+    code = ctypes.c_uint(0)
+    rc = load().fa_device_status(ctypes.byref(code))
+    if rc not in (0, -5):
+        _check(rc, "fa_device_status")
+    return int(code.value)

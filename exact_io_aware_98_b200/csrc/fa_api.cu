@@ -1,0 +1,311 @@
+// fa_api.cu -- the C ABI of libfa (declared in include/fa.h): argument validation, TMA
+// tensor-map encoding and kernel launches.  No allocation, no host synchronisation.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "fa.h"
+#include "fa_bwd_sm100.cuh"
+#include "fa_fwd_sm100.cuh"
+#include "fa_simt.cuh"
+#include "ptx.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return FA_OK;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qres) ==
+            cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D view [B*H][N][d] bf16 of a contiguous tensor, 128-byte swizzled boxes of 64 x rows.
+int make_map(CUtensorMap* map, const void* base, int BH, int N, int d, int box_rows,
+             const char* name) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(N) * d * 2};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "tensor map for %s failed (%d)", name, (int)r);
+  return FA_OK;
+}
+
+template <typename Kernel>
+int set_smem(Kernel kernel, int bytes) {
+  const cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(e));
+  return FA_OK;
+}
+
+int common_checks(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                  int B, int H, int N, int d, float scale) {
+  if (!q || !k || !v || !o || !lse) return fail(FA_ERR_INVALID, "null tensor pointer");
+  if (B < 1 || H < 1 || N < 1 || d < 1) return fail(FA_ERR_INVALID, "B, H, N, d must be >= 1");
+  if (!(std::isfinite(scale) && scale > 0.f)) return fail(FA_ERR_INVALID, "scale must be finite and > 0");
+  if (static_cast<long long>(B) * H > (1ll << 24)) return fail(FA_ERR_UNSUPPORTED, "B*H too large");
+  if (N > (1 << 24)) return fail(FA_ERR_UNSUPPORTED, "N too large");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return fail(FA_ERR_ALIGN, "tensor pointers must be 16-byte aligned");
+  return FA_OK;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct BwdWs {
+  size_t lse2, dvec, dq, total;
+  int n_pad;
+};
+BwdWs bwd_ws(int B, int H, int N, int d) {
+  BwdWs w;
+  w.n_pad = (N + 127) / 128 * 128;
+  const size_t bh = static_cast<size_t>(B) * H;
+  w.lse2 = 0;
+  w.dvec = round256(bh * w.n_pad * 4);
+  w.dq = w.dvec + round256(bh * w.n_pad * 4);
+  w.total = w.dq + round256(bh * static_cast<size_t>(N) * d * 4);
+  return w;
+}
+
+template <int D>
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int N, float scale, int causal, const uint8_t* bm, const int32_t* kv_len,
+               cudaStream_t stream) {
+  using L = fa::FwdLayout<D>;
+  CUtensorMap mq, mk, mv;
+  const int BH = B * H;
+  int rc;
+  if ((rc = make_map(&mq, q, BH, N, D, 128, "q")) != FA_OK) return rc;
+  if ((rc = make_map(&mk, k, BH, N, D, 128, "k")) != FA_OK) return rc;
+  if ((rc = make_map(&mv, v, BH, N, D, 128, "v")) != FA_OK) return rc;
+  if ((rc = set_smem(fa::fa_fwd_sm100_kernel<D>, L::SMEM_ALLOC)) != FA_OK) return rc;
+  fa::FwdParams p;
+  p.block_mask = bm;
+  p.kv_len = kv_len;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.n_mtiles = (N + 255) / 256;
+  p.scale2 = scale * kLog2e;
+  p.causal = causal ? 1 : 0;
+  const long long grid = static_cast<long long>(p.n_mtiles) * BH;
+  if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
+  fa::fa_fwd_sm100_kernel<D><<<static_cast<unsigned>(grid), 320, L::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
+  return check_launch("fa_fwd_sm100_kernel");
+}
+
+template <int D>
+int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+               int B, int H, int N, float scale, int causal, const uint8_t* bm,
+               const int32_t* kv_len, const BwdWs& ws, uint8_t* wsb, cudaStream_t stream) {
+  using L = fa::BwdLayout<D>;
+  CUtensorMap mq, mk, mv, mdo;
+  const int BH = B * H;
+  int rc;
+  if ((rc = make_map(&mq, q, BH, N, D, L::BM, "q")) != FA_OK) return rc;
+  if ((rc = make_map(&mk, k, BH, N, D, 128, "k")) != FA_OK) return rc;
+  if ((rc = make_map(&mv, v, BH, N, D, 128, "v")) != FA_OK) return rc;
+  if ((rc = make_map(&mdo, dO, BH, N, D, L::BM, "dO")) != FA_OK) return rc;
+  if ((rc = set_smem(fa::fa_bwd_sm100_kernel<D>, L::SMEM_ALLOC)) != FA_OK) return rc;
+  fa::BwdParams p;
+  p.block_mask = bm;
+  p.kv_len = kv_len;
+  p.lse2 = reinterpret_cast<const float*>(wsb + ws.lse2);
+  p.dvec = reinterpret_cast<const float*>(wsb + ws.dvec);
+  p.dq_acc = reinterpret_cast<float*>(wsb + ws.dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.N_pad = ws.n_pad;
+  p.n_ktiles = (N + 127) / 128;
+  p.scale = scale;
+  p.scale2 = scale * kLog2e;
+  p.causal = causal ? 1 : 0;
+  const long long grid = static_cast<long long>(p.n_ktiles) * BH;
+  if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
+  fa::fa_bwd_sm100_kernel<D><<<static_cast<unsigned>(grid), 320, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
+  return check_launch("fa_bwd_sm100_kernel");
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_get_last_error(void) { return g_err; }
+
+int fa_device_status(unsigned int* code) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "device synchronise: %s", cudaGetErrorString(e));
+  unsigned int v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, fa::g_status, sizeof(v));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(fa::g_status, &zero, sizeof(zero));
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "status word: %s", cudaGetErrorString(e));
+  if (code) *code = v;
+  if (v != 0) return fail(FA_ERR_TIMEOUT, "device wait gave up: site %u block %u", v >> 16, v & 0xffffu);
+  return FA_OK;
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+           int N, int d, float scale, int causal, const uint8_t* block_mask,
+           const int32_t* kv_len, int dtype, void* stream) {
+  int rc = common_checks(q, k, v, o, lse, B, H, N, d, scale);
+  if (rc != FA_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == FA_BF16) {
+    if (d == 64) return launch_fwd<64>(q, k, v, o, lse, B, H, N, scale, causal, block_mask, kv_len, s);
+    if (d == 128) return launch_fwd<128>(q, k, v, o, lse, B, H, N, scale, causal, block_mask, kv_len, s);
+    return fail(FA_ERR_UNSUPPORTED, "bf16 forward supports d in {64, 128}, got %d", d);
+  }
+  if (dtype == FA_F32) {
+    if (d > 128) return fail(FA_ERR_UNSUPPORTED, "fp32 forward supports d <= 128, got %d", d);
+    const long long rows = static_cast<long long>(B) * H * N;
+    fa::fa_fwd_rowwarp_kernel<float, false><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
+        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+        static_cast<float*>(o), lse, block_mask, kv_len, B, H, N, d, scale, causal ? 1 : 0, 128);
+    return check_launch("fa_fwd_rowwarp_kernel<f32>");
+  }
+  return fail(FA_ERR_INVALID, "unknown dtype %d", dtype);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
+  return bwd_ws(B, H, N, d).total;
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+           float scale, int causal, const uint8_t* block_mask, const int32_t* kv_len,
+           int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = common_checks(q, k, v, o, lse, B, H, N, d, scale);
+  if (rc != FA_OK) return rc;
+  if (!dO || !dq || !dk || !dv) return fail(FA_ERR_INVALID, "null gradient pointer");
+  if (!aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return fail(FA_ERR_ALIGN, "gradient pointers must be 16-byte aligned");
+  if (dtype != FA_BF16) {
+    if (dtype == FA_F32) return fail(FA_ERR_UNSUPPORTED, "fp32 backward is not built");
+    return fail(FA_ERR_INVALID, "unknown dtype %d", dtype);
+  }
+  if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "bf16 backward supports d in {64, 128}, got %d", d);
+  const BwdWs ws = bwd_ws(B, H, N, d);
+  if (workspace == nullptr || workspace_bytes < ws.total)
+    return fail(FA_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", ws.total, workspace_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(FA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  const int BH = B * H;
+  const long long pre_rows = static_cast<long long>(BH) * ws.n_pad;
+  fa::bwd_preprocess_kernel<<<static_cast<unsigned>((pre_rows + 7) / 8), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse,
+      reinterpret_cast<float*>(wsb + ws.lse2), reinterpret_cast<float*>(wsb + ws.dvec),
+      reinterpret_cast<float*>(wsb + ws.dq), BH, N, ws.n_pad, d);
+  if ((rc = check_launch("bwd_preprocess_kernel")) != FA_OK) return rc;
+  if (d == 64)
+    rc = launch_bwd<64>(q, k, v, dO, dk, dv, B, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+  else
+    rc = launch_bwd<128>(q, k, v, dO, dk, dv, B, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+  if (rc != FA_OK) return rc;
+  const long long n = static_cast<long long>(BH) * N * d;
+  fa::dq_convert_kernel<<<static_cast<unsigned>((n / 8 + 255) / 256 + 1), 256, 0, s>>>(
+      reinterpret_cast<const float*>(wsb + ws.dq), static_cast<__nv_bfloat16*>(dq), n, scale);
+  return check_launch("dq_convert_kernel");
+}
+
+int fa_fwd_tile_reference(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int H, int N, int d, float scale, int causal,
+                          const uint8_t* block_mask, const int32_t* kv_len, int bc,
+                          void* stream) {
+  int rc = common_checks(q, k, v, o, lse, B, H, N, d, scale);
+  if (rc != FA_OK) return rc;
+  if (d > 128) return fail(FA_ERR_UNSUPPORTED, "d <= 128 required, got %d", d);
+  if (bc < 32 || bc > 256 || (bc % 32) != 0) return fail(FA_ERR_INVALID, "bc must be 32..256 in steps of 32");
+  const long long rows = static_cast<long long>(B) * H * N;
+  fa::fa_fwd_rowwarp_kernel<__nv_bfloat16, true>
+      <<<static_cast<unsigned>((rows + 7) / 8), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+          static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+          static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), lse, block_mask,
+          kv_len, B, H, N, d, scale, causal ? 1 : 0, bc);
+  return check_launch("fa_fwd_rowwarp_kernel<bf16>");
+}
+
+size_t fa_naive_workspace_size(int B, int H, int N) {
+  if (B < 1 || H < 1 || N < 1) return 0;
+  return static_cast<size_t>(B) * H * N * N * 2;
+}
+
+int fa_naive_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, float scale, int causal, const uint8_t* block_mask,
+                 const int32_t* kv_len, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = common_checks(q, k, v, o, lse, B, H, N, d, scale);
+  if (rc != FA_OK) return rc;
+  if (d > 128) return fail(FA_ERR_UNSUPPORTED, "d <= 128 required, got %d", d);
+  const size_t need = fa_naive_workspace_size(B, H, N);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(FA_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", need, workspace_bytes);
+  if (N > 65535 * 16) return fail(FA_ERR_UNSUPPORTED, "N too large for the naive kernel");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  if (BH > 65535) return fail(FA_ERR_UNSUPPORTED, "B*H too large for the naive kernel");
+  __nv_bfloat16* sm = static_cast<__nv_bfloat16*>(workspace);
+  const dim3 g1((N + 15) / 16, (N + 15) / 16, BH);
+  fa::naive_scores_kernel<<<g1, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(q),
+                                             static_cast<const __nv_bfloat16*>(k), sm, block_mask,
+                                             kv_len, H, N, d, scale, causal ? 1 : 0);
+  if ((rc = check_launch("naive_scores_kernel")) != FA_OK) return rc;
+  const long long rows = static_cast<long long>(BH) * N;
+  fa::naive_softmax_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(sm, lse, rows, N);
+  if ((rc = check_launch("naive_softmax_kernel")) != FA_OK) return rc;
+  const dim3 g3(1, (N + 15) / 16, BH);
+  fa::naive_pv_kernel<<<g3, 256, 0, s>>>(sm, static_cast<const __nv_bfloat16*>(v),
+                                         static_cast<__nv_bfloat16*>(o), N, d);
+  return check_launch("naive_pv_kernel");
+}
+
+}  // extern "C"

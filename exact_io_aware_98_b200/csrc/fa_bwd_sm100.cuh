@@ -1,0 +1,442 @@
+// fa_bwd_sm100.cuh -- exact attention backward on sm_100a, recomputing the scores from Q, K
+// and the forward's per-row log-sum-exp (no N x N matrix is stored).
+//
+// Derivative of O = softmax(S) V with S = scale * Q K^T (the formula of "Attention
+// optimisation: FlashAttention and sparse attention", mdooai Ch.04), written with
+// Dvec_i = sum_c dO_ic O_ic, which equals sum_k A_ik dA_ik because O = A V:
+//   P_ij  = 2^(s_ij * scale2 - lse_i * log2 e)            (= A_ij; 0 for masked keys)
+//   dV_j  = sum_i P_ij dO_i
+//   dP_ij = dO_i . v_j
+//   dS_ij = P_ij (dP_ij - Dvec_i)
+//   dK_j  = scale * sum_i dS_ij q_i
+//   dQ_i  = scale * sum_j dS_ij k_j
+//
+// One CTA owns 128 keys (K and V stay in shared memory) and walks the query tiles that can
+// see them (causal, key padding and block mask skip whole tiles).  Per query tile of BM rows:
+//   S^T  = K Q^T     (M=128 keys, N=BM, K=D)      smem x smem  -> TMEM
+//   dP^T = V dO^T    (M=128, N=BM, K=D)           smem x smem  -> TMEM
+//   compute warpgroup: P^T, dS^T in bf16 back into TMEM (over S^T / dP^T) and dS^T to smem
+//   dV  += P^T dO    (M=128, N=D, K=BM)           TMEM x smem  -> TMEM
+//   dK  += dS^T Q    (M=128, N=D, K=BM)           TMEM x smem  -> TMEM
+//   D=64 : dQ   = dS K     (M=BM=128, N=64,  K=128) smem x smem -> TMEM (row per lane)
+//   D=128: dQ^T = K^T dS^T (M=128,    N=BM=64, K=128) smem x smem -> TMEM (column per lane)
+//   dQ warpgroup: TMEM -> fp32 red.global.add into the dQ workspace.
+// The MMA thread issues dV(t), S(t+1), dK(t), dP(t+1), dQ(t): in-order execution lets S(t+1)
+// reuse the TMEM that dV(t) read P^T(t) from, and dP(t+1) the TMEM of dS^T(t), so the
+// compute warpgroup works on step t+1 while dQ(t) runs.
+//
+// CTA: 320 threads. warps 0-3 compute, warp 4 TMA producer, warp 5 MMA issuer, warps 6-9 dQ.
+#pragma once
+#include "ptx.cuh"
+
+namespace fa {
+
+struct BwdParams {
+  const uint8_t* block_mask;  // [nb][nb] or nullptr
+  const int32_t* kv_len;      // [B] or nullptr
+  const float* lse2;          // [B*H][N_pad] lse*log2(e); +inf for rows with no key / padding
+  const float* dvec;          // [B*H][N_pad]
+  float* dq_acc;              // [B*H][N][D] fp32, zeroed by the preprocess kernel
+  __nv_bfloat16* dk;          // [B*H][N][D]
+  __nv_bfloat16* dv;          // [B*H][N][D]
+  int B, H, N, N_pad;
+  int n_ktiles;               // ceil(N / 128)
+  float scale, scale2;
+  int causal;
+};
+
+template <int D>
+struct BwdLayout {
+  static constexpr int BN = 128;                  // keys per CTA
+  static constexpr int BM = D == 64 ? 128 : 64;   // query rows per step
+  static constexpr int QST = 2;
+  static constexpr int SUB = D / 64;
+  static constexpr int KV_SUBTILE = 128 * 128;
+  static constexpr int Q_SUBTILE = BM * 128;
+  static constexpr int KV_TILE = 128 * D * 2;
+  static constexpr int Q_TILE = BM * D * 2;
+  static constexpr int DS_TILE = BN * BM * 2;     // dS^T rows j, 64-column i-blocks
+  static constexpr int DS_IBLK = BN * 128;        // bytes between i-blocks of dS^T
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KV_TILE;
+  static constexpr int OFF_Q = OFF_V + KV_TILE;
+  static constexpr int OFF_DO = OFF_Q + QST * Q_TILE;
+  static constexpr int OFF_DS = OFF_DO + QST * Q_TILE;
+  static constexpr int OFF_LSE = OFF_DS + 2 * DS_TILE;
+  static constexpr int OFF_DVEC = OFF_LSE + QST * BM * 4;
+  static constexpr int OFF_BAR = OFF_DVEC + QST * BM * 4;
+  // kv, q_full[QST], q_empty[QST], sdp_full, ds_full, dq_full[2], dq_empty[2], kv_done, fin
+  static constexpr int NBAR = 1 + 2 * QST + 1 + 1 + 2 + 2 + 1 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int SMEM_ALLOC = BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t S_COL = 0;
+  static constexpr uint32_t DP_COL = BM;
+  static constexpr uint32_t DQ_COL = 2 * BM;           // two 64-column buffers
+  static constexpr uint32_t DV_COL = 2 * BM + 128;
+  static constexpr uint32_t DK_COL = 2 * BM + 128 + D;
+  static_assert(DK_COL + D <= TMEM_COLS, "TMEM budget");
+};
+
+enum : int {
+  SITE_BWD_LOAD_EMPTY = 21, SITE_BWD_LOAD_DRAIN = 22, SITE_BWD_MMA_KV = 23, SITE_BWD_MMA_Q = 24,
+  SITE_BWD_MMA_DS = 25, SITE_BWD_MMA_DQE = 26, SITE_BWD_MMA_FIN = 27, SITE_BWD_C_Q = 28,
+  SITE_BWD_C_SDP = 29, SITE_BWD_C_DQ = 30, SITE_BWD_C_DONE = 31, SITE_BWD_DQ = 32
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+  using L = BwdLayout<D>;
+  constexpr int BM = L::BM;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* bar_kv = bars;
+  uint64_t* bar_qf = bars + 1;
+  uint64_t* bar_qe = bar_qf + L::QST;
+  uint64_t* bar_sdp = bar_qe + L::QST;
+  uint64_t* bar_ds = bar_sdp + 1;
+  uint64_t* bar_dqf = bar_ds + 1;
+  uint64_t* bar_dqe = bar_dqf + 2;
+  uint64_t* bar_done = bar_dqe + 2;
+  uint64_t* bar_fin = bar_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+  const float* s_lse = reinterpret_cast<const float*>(smem + L::OFF_LSE);
+  const float* s_dvec = reinterpret_cast<const float*>(smem + L::OFF_DVEC);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int BH = p.B * p.H;
+  const int jt = static_cast<int>(blockIdx.x) / BH;  // KV tile; small jt (most work) first
+  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int b = bh / p.H;
+  const int N = p.N;
+  const int k0 = jt * 128;
+  int kvlen = N;
+  if (p.kv_len != nullptr) kvlen = min(max(p.kv_len[b], 0), N);
+  const int nb = (N + 127) / 128;
+  const int n_qt = (N + BM - 1) / BM;
+  const bool kv_live = k0 < kvlen;
+
+  // query tile `it` (rows it*BM ..) has at least one (row, key) pair with this KV tile
+  auto q_active = [&](int it) -> bool {
+    if (!kv_live) return false;
+    const int i0 = it * BM;
+    if (p.causal && i0 + BM - 1 < k0) return false;
+    if (p.block_mask != nullptr && !p.block_mask[static_cast<size_t>(i0 >> 7) * nb + jt])
+      return false;
+    return true;
+  };
+  int n_steps = 0;
+  for (int it = 0; it < n_qt; ++it) n_steps += q_active(it) ? 1 : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_kv, 1);
+    for (int s = 0; s < L::QST; ++s) {
+      mbar_init(&bar_qf[s], 1);
+      mbar_init(&bar_qe[s], 1);
+    }
+    mbar_init(bar_sdp, 1);
+    mbar_init(bar_ds, 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_dqf[i], 1);
+      mbar_init(&bar_dqe[i], 128);
+    }
+    mbar_init(bar_done, 1);
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && n_steps > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(bar_kv, 2 * L::KV_TILE);
+      for (int s = 0; s < L::SUB; ++s) {
+        tma_load_3d(smem + L::OFF_K + s * L::KV_SUBTILE, &tm_k, bar_kv, s * 64, k0, bh);
+        tma_load_3d(smem + L::OFF_V + s * L::KV_SUBTILE, &tm_v, bar_kv, s * 64, k0, bh);
+      }
+      int t = 0;
+      for (int it = 0; it < n_qt; ++it) {
+        if (!q_active(it)) continue;
+        const int st = t % L::QST;
+        if (t >= L::QST &&
+            !mbar_wait(&bar_qe[st], ((t / L::QST) - 1) & 1, abort_flag, SITE_BWD_LOAD_EMPTY))
+          break;
+        const int i0 = it * BM;
+        mbar_arrive_expect_tx(&bar_qf[st], 2 * L::Q_TILE + 2 * BM * 4);
+        for (int s = 0; s < L::SUB; ++s) {
+          tma_load_3d(smem + L::OFF_Q + st * L::Q_TILE + s * L::Q_SUBTILE, &tm_q, &bar_qf[st],
+                      s * 64, i0, bh);
+          tma_load_3d(smem + L::OFF_DO + st * L::Q_TILE + s * L::Q_SUBTILE, &tm_do, &bar_qf[st],
+                      s * 64, i0, bh);
+        }
+        const size_t off = static_cast<size_t>(bh) * p.N_pad + i0;
+        bulk_load(smem + L::OFF_LSE + st * BM * 4, p.lse2 + off, BM * 4, &bar_qf[st]);
+        bulk_load(smem + L::OFF_DVEC + st * BM * 4, p.dvec + off, BM * 4, &bar_qf[st]);
+        ++t;
+      }
+      mbar_wait(bar_kv, 0, abort_flag, SITE_BWD_LOAD_DRAIN);
+      for (int r = max(0, t - L::QST); r < t; ++r)
+        mbar_wait(&bar_qf[r % L::QST], (r / L::QST) & 1, abort_flag, SITE_BWD_LOAD_DRAIN);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_steps > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, BM, false, false);
+      constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t idesc_q = idesc_bf16_f32(128, 64, true, true);
+      const uint32_t k_addr = smem_u32(smem + L::OFF_K);
+      const uint32_t v_addr = smem_u32(smem + L::OFF_V);
+      const uint32_t q_addr = smem_u32(smem + L::OFF_Q);
+      const uint32_t do_addr = smem_u32(smem + L::OFF_DO);
+      const uint32_t ds_addr = smem_u32(smem + L::OFF_DS);
+      // X^T = A B^T over D: A = K or V tile (128 rows), B = Q or dO tile (BM rows), K-major.
+      auto mma_scores = [&](uint32_t a_base, uint32_t b_base, uint32_t d_col) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const int sub = k >> 2, kk = k & 3;
+          const uint64_t ad = sdesc_sw128(a_base + sub * L::KV_SUBTILE + kk * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(b_base + sub * L::Q_SUBTILE + kk * 32, 16, 1024);
+          mma_ss(tmem + d_col, ad, bd, idesc_s, k > 0 ? 1u : 0u);
+        }
+      };
+      // G += X^T(TMEM, bf16) B over BM rows: B = dO or Q tile, MN-major.
+      auto mma_grad = [&](uint32_t a_col, uint32_t b_base, uint32_t d_col, bool acc) {
+#pragma unroll
+        for (int k = 0; k < BM / 16; ++k) {
+          const uint64_t bd = sdesc_sw128(b_base + k * 2048, L::Q_SUBTILE, 1024);
+          mma_ts(tmem + d_col, tmem + a_col + k * 8, bd, idesc_g, (acc || k > 0) ? 1u : 0u);
+        }
+      };
+      auto mma_dq = [&](int buf) {
+        const uint32_t ds = ds_addr + buf * L::DS_TILE;
+#pragma unroll
+        for (int k = 0; k < L::BN / 16; ++k) {
+          uint64_t ad, bd;
+          if constexpr (D == 64) {  // dQ = dS K: A = dS (i contiguous), B = K (d contiguous)
+            ad = sdesc_sw128(ds + k * 2048, L::DS_IBLK, 1024);
+            bd = sdesc_sw128(k_addr + k * 2048, L::KV_SUBTILE, 1024);
+          } else {                  // dQ^T = K^T dS^T: A = K^T (d contiguous), B = dS^T
+            ad = sdesc_sw128(k_addr + k * 2048, L::KV_SUBTILE, 1024);
+            bd = sdesc_sw128(ds + k * 2048, L::DS_IBLK, 1024);
+          }
+          mma_ss(tmem + L::DQ_COL + buf * 64, ad, bd, idesc_q, k > 0 ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(bar_kv, 0, abort_flag, SITE_BWD_MMA_KV);
+      ok = ok && mbar_wait(&bar_qf[0], 0, abort_flag, SITE_BWD_MMA_Q);
+      tc_fence_after();
+      if (ok) {
+        mma_scores(k_addr, q_addr, L::S_COL);
+        mma_scores(v_addr, do_addr, L::DP_COL);
+        mma_commit(bar_sdp);
+      }
+      for (int t = 0; ok && t < n_steps; ++t) {
+        const int st = t % L::QST;
+        const int buf = t & 1;
+        if (!mbar_wait(bar_ds, t & 1, abort_flag, SITE_BWD_MMA_DS)) { ok = false; break; }
+        tc_fence_after();
+        mma_grad(L::S_COL, do_addr + st * L::Q_TILE, L::DV_COL, t > 0);
+        const bool next = t + 1 < n_steps;
+        const int st1 = (t + 1) % L::QST;
+        if (next) {
+          if (!mbar_wait(&bar_qf[st1], ((t + 1) / L::QST) & 1, abort_flag, SITE_BWD_MMA_Q)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_scores(k_addr, q_addr + st1 * L::Q_TILE, L::S_COL);
+        }
+        mma_grad(L::DP_COL, q_addr + st * L::Q_TILE, L::DK_COL, t > 0);
+        if (next) {
+          mma_scores(v_addr, do_addr + st1 * L::Q_TILE, L::DP_COL);
+          mma_commit(bar_sdp);
+        }
+        if (t >= 2 && !mbar_wait(&bar_dqe[buf], ((t - 2) >> 1) & 1, abort_flag, SITE_BWD_MMA_DQE)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        mma_dq(buf);
+        mma_commit(&bar_dqf[buf]);
+        mma_commit(&bar_qe[st]);
+      }
+      mma_commit(bar_done);
+      mma_commit(bar_fin);
+      mbar_wait(bar_fin, 0, abort_flag, SITE_BWD_MMA_FIN);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------------ compute warpgroup
+    const int qw = warp & 3;
+    const int jl = 32 * qw + lane;            // key row within the tile (= TMEM lane)
+    const int kj = k0 + jl;                   // key index
+    const uint32_t t_lane = static_cast<uint32_t>(32 * qw) << 16;
+    const float scale2 = p.scale2;
+    bool ok = true;
+    int t = 0;
+    for (int it = 0; it < n_qt; ++it) {
+      if (!q_active(it)) continue;
+      const int st = t % L::QST;
+      const int buf = t & 1;
+      const int i0 = it * BM;
+      bool got = mbar_wait(&bar_qf[st], (t / L::QST) & 1, abort_flag, SITE_BWD_C_Q);
+      got = got && mbar_wait(bar_sdp, t & 1, abort_flag, SITE_BWD_C_SDP);
+      if (t >= 2) got = got && mbar_wait(&bar_dqf[buf], ((t - 2) >> 1) & 1, abort_flag, SITE_BWD_C_DQ);
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      tc_fence_after();
+      const float* lse_s = s_lse + st * BM;
+      const float* dv_s = s_dvec + st * BM;
+      const bool edge = (k0 + 128 > kvlen) || (p.causal && k0 + 32 * qw + 31 > i0);
+      uint8_t* ds_row = smem + L::OFF_DS + buf * L::DS_TILE + jl * 128;
+#pragma unroll 1
+      for (int cc = 0; cc < BM / 32; ++cc) {
+        uint32_t s[32], dp[32];
+        tmem_ld32(tmem + t_lane + L::S_COL + 32 * cc, s);
+        tmem_ld32(tmem + t_lane + L::DP_COL + 32 * cc, dp);
+        tmem_ld_wait();
+        reg_fence(s);
+        reg_fence(dp);
+        uint32_t pp[16], dd[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float pv[2], dsv[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int col = 32 * cc + 2 * i + h;
+            float pe = ex2_approx(fmaf(__uint_as_float(s[2 * i + h]), scale2, -lse_s[col]));
+            if (edge && (kj >= kvlen || (p.causal && kj > i0 + col))) pe = 0.f;
+            pv[h] = pe;
+            dsv[h] = pe * (__uint_as_float(dp[2 * i + h]) - dv_s[col]);
+          }
+          pp[i] = pack_bf16x2(pv[0], pv[1]);
+          dd[i] = pack_bf16x2(dsv[0], dsv[1]);
+        }
+        tmem_st16(tmem + t_lane + L::S_COL + 16 * cc, pp);
+        tmem_st16(tmem + t_lane + L::DP_COL + 16 * cc, dd);
+        // dS^T row jl, columns 32cc..32cc+31 -> 4 swizzled 16-byte chunks
+        const int iblk = (32 * cc) >> 6;
+        const int chunk0 = ((32 * cc) & 63) >> 3;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int pos = (chunk0 + u) ^ (jl & 7);
+          *reinterpret_cast<uint4*>(ds_row + iblk * L::DS_IBLK + pos * 16) =
+              make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
+        }
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_ds);
+      ++t;
+    }
+    // ---------------------------------------------------------------- epilogue: dK, dV
+    if (ok && n_steps > 0) {
+      const bool got = mbar_wait(bar_done, 0, abort_flag, SITE_BWD_C_DONE);
+      ok = __all_sync(0xffffffffu, got);
+      tc_fence_after();
+    }
+    if (ok && k0 < N) {
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col0 = which == 0 ? L::DV_COL : L::DK_COL;
+        const float mul = which == 0 ? 1.0f : p.scale;
+        __nv_bfloat16* dst_row =
+            (which == 0 ? p.dv : p.dk) + (static_cast<size_t>(bh) * N + kj) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t g[32];
+          if (n_steps > 0) {
+            tmem_ld32(tmem + t_lane + col0 + 32 * c, g);
+            tmem_ld_wait();
+            reg_fence(g);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) g[i] = 0u;
+          }
+          uint32_t h[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            h[i] = pack_bf16x2(__uint_as_float(g[2 * i]) * mul, __uint_as_float(g[2 * i + 1]) * mul);
+          if (kj < N) {
+            uint4* dst = reinterpret_cast<uint4*>(dst_row + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ dQ warpgroup
+    const int qw = warp & 3;
+    const uint32_t t_lane = static_cast<uint32_t>(32 * qw) << 16;
+    int t = 0;
+    for (int it = 0; it < n_qt; ++it) {
+      if (!q_active(it)) continue;
+      const int buf = t & 1;
+      const int i0 = it * BM;
+      const bool got = mbar_wait(&bar_dqf[buf], (t >> 1) & 1, abort_flag, SITE_BWD_DQ);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      uint32_t v[2][32];
+      tmem_ld32(tmem + t_lane + L::DQ_COL + buf * 64, v[0]);
+      tmem_ld32(tmem + t_lane + L::DQ_COL + buf * 64 + 32, v[1]);
+      tmem_ld_wait();
+      reg_fence(v[0]);
+      reg_fence(v[1]);
+      tc_fence_before();
+      mbar_arrive(&bar_dqe[buf]);
+      if constexpr (D == 64) {
+        // lane = query row i0 + 32qw + lane, 64 columns of dQ
+        const int qi = i0 + 32 * qw + lane;
+        if (qi < N) {
+          float4* dst = reinterpret_cast<float4*>(p.dq_acc + (static_cast<size_t>(bh) * N + qi) * D);
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const uint32_t* src = &v[u >> 3][(u & 7) * 4];
+            atomicAdd(dst + u, make_float4(__uint_as_float(src[0]), __uint_as_float(src[1]),
+                                           __uint_as_float(src[2]), __uint_as_float(src[3])));
+          }
+        }
+      } else {
+        // lane = head dimension c, columns = query rows i0 .. i0+63
+        const int c = 32 * qw + lane;
+        float* base = p.dq_acc + (static_cast<size_t>(bh) * N + i0) * D + c;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          if (i0 + i < N) atomicAdd(base + static_cast<size_t>(i) * D, __uint_as_float(v[i >> 5][i & 31]));
+        }
+      }
+      ++t;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+}  // namespace fa

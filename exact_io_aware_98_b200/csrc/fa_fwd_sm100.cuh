@@ -1,0 +1,394 @@
+// fa_fwd_sm100.cuh -- exact attention forward on sm_100a: TMA-fed tiles, tcgen05 MMAs with
+// TMEM accumulators, online softmax in warp-specialised warpgroups.
+//
+// Computes, per (b, h): S = scale * Q K^T with masked keys at -inf, A = row softmax of S,
+// O = A V, and the per-row log-sum-exp of S ("Attention optimisation: FlashAttention and
+// sparse attention", mdooai Ch.04, core formula and the sparse-masking paragraph), without
+// ever writing S or A to HBM: the five stages of "What is FlashAttention? Why smarter memory
+// use speeds up transformers" (tile Q/K/V; load small blocks on chip; local scores with a
+// running normalisation; accumulate the output without materialising the full matrix;
+// schedule for the target accelerator).
+//
+// CTA layout (320 threads, one CTA per SM):
+//   warps 0-3  softmax warpgroup for Q tile 0 (rows m0 .. m0+127), one thread per row
+//   warps 4-7  softmax warpgroup for Q tile 1 (rows m0+128 .. m0+255)
+//   warp  8    TMA producer: Q once, then K/V tiles of 128 keys through a STAGES-deep ring
+//   warp  9    MMA issuer (one thread): S_w = Q_w K^T into TMEM, O_w += P_w V from TMEM P
+// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [256+D,256+2D).
+// P_w (bf16, two per 32-bit column) overwrites columns [0,64) of S_w after the softmax
+// warpgroup has read S_w into registers.
+//
+// Per KV tile the MMA thread issues, for w = 0 then 1: PV_w of the previous tile, then S_w of
+// this tile.  tcgen05 MMAs from one thread execute in issue order, so S_w(t+1) cannot overwrite
+// P_w(t) before PV_w(t) has read it, and the commit that signals S_w(t+1) also certifies that
+// PV_w(t) has finished -- which is what lets a softmax warpgroup rescale O_w right after it
+// sees S_w(t+1), with no extra barrier.
+//
+// Online softmax (log2 domain, scale2 = scale*log2 e): the running reference m is raised only
+// when a tile's maximum exceeds it by more than 8 (a factor 256); O and l are then multiplied
+// by 2^(m_old - m_new).  P = 2^(s*scale2 - m) <= 256 and l accumulate exactly as with an
+// always-updated maximum, and the final O/l and lse = (m + log2 l) ln 2 use the same m, so the
+// result is the same softmax.
+#pragma once
+#include "ptx.cuh"
+
+namespace fa {
+
+struct FwdParams {
+  const uint8_t* block_mask;  // [nb][nb] (nb = ceil(N/128)) or nullptr
+  const int32_t* kv_len;      // [B] or nullptr
+  __nv_bfloat16* o;           // [B*H][N][D]
+  float* lse;                 // [B*H][N]
+  int B, H, N;
+  int n_mtiles;               // ceil(N / 256)
+  float scale2;               // scale * log2(e)
+  int causal;
+};
+
+template <int D>
+struct FwdLayout {
+  static constexpr int BM = 128;                    // query rows per Q tile
+  static constexpr int BN = 128;                    // keys per KV tile
+  static constexpr int STAGES = D == 64 ? 4 : 2;
+  static constexpr int SUB = D / 64;                // 64-column (128-byte) sub-tiles
+  static constexpr int SUBTILE = 128 * 128;         // bytes of one 128-row x 64-col sub-tile
+  static constexpr int TILE = 128 * D * 2;          // bytes of one 128-row tile
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * TILE;
+  static constexpr int OFF_V = OFF_K + STAGES * TILE;
+  static constexpr int OFF_BAR = OFF_V + STAGES * TILE;
+  static constexpr int NBAR = 1 + 3 * STAGES + 6 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int SMEM_ALLOC = BYTES + 1024;   // slack for 1024-byte alignment
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t O_COL0 = 256;
+  __device__ static constexpr uint32_t s_col(int w) { return static_cast<uint32_t>(w) * 128u; }
+};
+
+// Wait-site codes recorded in the status word on a timeout.
+enum : int {
+  SITE_FWD_LOAD_EMPTY = 1, SITE_FWD_LOAD_DRAIN = 2, SITE_FWD_MMA_Q = 3, SITE_FWD_MMA_K = 4,
+  SITE_FWD_MMA_V = 5, SITE_FWD_MMA_P = 6, SITE_FWD_MMA_FIN = 7, SITE_FWD_SM_S = 8,
+  SITE_FWD_SM_O = 9
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using L = FwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_kf = bars + 1;
+  uint64_t* bar_vf = bar_kf + L::STAGES;
+  uint64_t* bar_ke = bar_vf + L::STAGES;
+  uint64_t* bar_sf = bar_ke + L::STAGES;
+  uint64_t* bar_pf = bar_sf + 2;
+  uint64_t* bar_od = bar_pf + 2;
+  uint64_t* bar_fin = bar_od + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int BH = p.B * p.H;
+  const int mt = p.n_mtiles - 1 - static_cast<int>(blockIdx.x) / BH;  // heaviest tiles first
+  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int b = bh / p.H;
+  const int N = p.N;
+  const int m0 = mt * 256;
+  int kvlen = N;
+  if (p.kv_len != nullptr) kvlen = min(max(p.kv_len[b], 0), N);
+  const int nb = (N + 127) / 128;
+  const int n_kv = (kvlen + 127) / 128;
+  int j_end = n_kv;
+  if (p.causal) j_end = min(j_end, (min(m0 + 256, N) - 1) / 128 + 1);
+
+  // bit w set: KV tile j holds at least one key that Q tile w may attend to
+  auto flags_of = [&](int j) -> int {
+    int f = 0;
+    const int k0 = j * 128;
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      const int q0 = m0 + 128 * w;
+      if (q0 >= N) continue;
+      const int q1 = min(q0 + 127, N - 1);
+      if (p.causal && k0 > q1) continue;
+      if (p.block_mask != nullptr && !p.block_mask[static_cast<size_t>(q0 >> 7) * nb + j]) continue;
+      f |= 1 << w;
+    }
+    return f;
+  };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < L::STAGES; ++s) {
+      mbar_init(&bar_kf[s], 1);
+      mbar_init(&bar_vf[s], 1);
+      mbar_init(&bar_ke[s], 1);
+    }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&bar_sf[w], 1);
+      mbar_init(&bar_pf[w], 128);
+      mbar_init(&bar_od[w], 1);
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const int nq = (m0 + 128 < N) ? 2 : 1;
+      mbar_arrive_expect_tx(bar_q, nq * L::TILE);
+      for (int w = 0; w < nq; ++w)
+        for (int s = 0; s < L::SUB; ++s)
+          tma_load_3d(smem + L::OFF_Q + w * L::TILE + s * L::SUBTILE, &tm_q, bar_q, s * 64,
+                      m0 + 128 * w, bh);
+      int it = 0;
+      for (int j = 0; j < j_end; ++j) {
+        if (flags_of(j) == 0) continue;
+        const int st = it % L::STAGES;
+        if (it >= L::STAGES &&
+            !mbar_wait(&bar_ke[st], ((it / L::STAGES) - 1) & 1, abort_flag, SITE_FWD_LOAD_EMPTY))
+          break;
+        mbar_arrive_expect_tx(&bar_kf[st], L::TILE);
+        for (int s = 0; s < L::SUB; ++s)
+          tma_load_3d(smem + L::OFF_K + st * L::TILE + s * L::SUBTILE, &tm_k, &bar_kf[st], s * 64,
+                      j * 128, bh);
+        mbar_arrive_expect_tx(&bar_vf[st], L::TILE);
+        for (int s = 0; s < L::SUB; ++s)
+          tma_load_3d(smem + L::OFF_V + st * L::TILE + s * L::SUBTILE, &tm_v, &bar_vf[st], s * 64,
+                      j * 128, bh);
+        ++it;
+      }
+      // Never leave the CTA with a copy in flight: wait for the last loads of every stage
+      // (immediate in the normal path, where the MMA thread consumed them).
+      mbar_wait(bar_q, 0, abort_flag, SITE_FWD_LOAD_DRAIN);
+      for (int r = max(0, it - L::STAGES); r < it; ++r) {
+        mbar_wait(&bar_kf[r % L::STAGES], (r / L::STAGES) & 1, abort_flag, SITE_FWD_LOAD_DRAIN);
+        mbar_wait(&bar_vf[r % L::STAGES], (r / L::STAGES) & 1, abort_flag, SITE_FWD_LOAD_DRAIN);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+      const uint32_t q_addr = smem_u32(smem + L::OFF_Q);
+      const uint32_t k_addr = smem_u32(smem + L::OFF_K);
+      const uint32_t v_addr = smem_u32(smem + L::OFF_V);
+      bool ok = mbar_wait(bar_q, 0, abort_flag, SITE_FWD_MMA_Q);
+      tc_fence_after();
+      int it = 0;
+      int cnt[2] = {0, 0};
+      int prev_flags = 0, prev_st = 0;
+      auto issue_pv = [&](int w, int st) -> bool {
+        if (!mbar_wait(&bar_pf[w], cnt[w] & 1, abort_flag, SITE_FWD_MMA_P)) return false;
+        tc_fence_after();
+        const uint32_t a_tmem = tmem + L::s_col(w);
+        const uint32_t d_tmem = tmem + L::O_COL0 + w * D;
+#pragma unroll
+        for (int k = 0; k < L::BN / 16; ++k) {
+          const uint64_t bdesc =
+              sdesc_sw128(v_addr + st * L::TILE + k * 2048, L::SUBTILE, 1024);
+          mma_ts(d_tmem, a_tmem + k * 8, bdesc, idesc_o, (cnt[w] > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(&bar_od[w]);
+        ++cnt[w];
+        return true;
+      };
+      for (int j = 0; ok && j < j_end; ++j) {
+        const int f = flags_of(j);
+        if (f == 0) continue;
+        const int st = it % L::STAGES;
+        if (!mbar_wait(&bar_kf[st], (it / L::STAGES) & 1, abort_flag, SITE_FWD_MMA_K)) { ok = false; break; }
+        if (prev_flags != 0 &&
+            !mbar_wait(&bar_vf[prev_st], ((it - 1) / L::STAGES) & 1, abort_flag, SITE_FWD_MMA_V)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          if (prev_flags & (1 << w)) {
+            if (!issue_pv(w, prev_st)) { ok = false; break; }
+          }
+          if (f & (1 << w)) {
+            const uint32_t d_tmem = tmem + L::s_col(w);
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              const int sub = k >> 2, kk = k & 3;
+              const uint64_t adesc =
+                  sdesc_sw128(q_addr + w * L::TILE + sub * L::SUBTILE + kk * 32, 16, 1024);
+              const uint64_t bdesc =
+                  sdesc_sw128(k_addr + st * L::TILE + sub * L::SUBTILE + kk * 32, 16, 1024);
+              mma_ss(d_tmem, adesc, bdesc, idesc_s, k > 0 ? 1u : 0u);
+            }
+            mma_commit(&bar_sf[w]);
+          }
+        }
+        if (!ok) break;
+        if (prev_flags != 0) mma_commit(&bar_ke[prev_st]);
+        prev_flags = f;
+        prev_st = st;
+        ++it;
+      }
+      if (ok && prev_flags != 0) {
+        if (mbar_wait(&bar_vf[prev_st], ((it - 1) / L::STAGES) & 1, abort_flag, SITE_FWD_MMA_V)) {
+          tc_fence_after();
+          for (int w = 0; w < 2; ++w)
+            if (prev_flags & (1 << w)) {
+              if (!issue_pv(w, prev_st)) break;
+            }
+          mma_commit(&bar_ke[prev_st]);
+        }
+      }
+      // all MMAs issued by this thread have completed before TMEM is released
+      mma_commit(bar_fin);
+      mbar_wait(bar_fin, 0, abort_flag, SITE_FWD_MMA_FIN);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int w = warp >> 2;
+    const int qw = warp & 3;
+    const int row_in_tile = 32 * qw + lane;
+    const int q0 = m0 + 128 * w;
+    const int row = q0 + row_in_tile;
+    const uint32_t t_lane = static_cast<uint32_t>(32 * qw) << 16;
+    const uint32_t t_s = tmem + t_lane + L::s_col(w);
+    const uint32_t t_o = tmem + t_lane + L::O_COL0 + w * D;
+    const float scale2 = p.scale2;
+    float m_ref = -INFINITY;  // running reference maximum (log2 domain, scaled)
+    float l = 0.f;            // running row sum of P
+    int cnt = 0;
+    bool ok = true;
+    for (int j = 0; j < j_end; ++j) {
+      if (!((flags_of(j) >> w) & 1)) continue;
+      const bool got = mbar_wait(&bar_sf[w], cnt & 1, abort_flag, SITE_FWD_SM_S);
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(t_s + 32 * c, r[c]);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence(r[c]);
+      const int k0 = j * 128;
+      const bool edge = (k0 + 128 > kvlen) || (p.causal && k0 + 127 > q0 + 32 * qw);
+      if (edge) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int col = k0 + 32 * c + i;
+            if (col >= kvlen || (p.causal && col > row)) r[c][i] = __float_as_uint(-INFINITY);
+          }
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(r[c][i]));
+      const float tmax = mx * scale2;
+      float m_new = m_ref;
+      if (tmax > m_ref + 8.0f) m_new = tmax;  // also taken when m_ref is still -inf
+      const float alpha = (m_new == m_ref) ? 1.0f : ex2_approx(m_ref - m_new);
+      const float neg_base = (m_new == -INFINITY) ? 0.0f : -m_new;
+      float rs0 = 0.f, rs1 = 0.f;
+      uint32_t pk[4][16];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][2 * i]), scale2, neg_base));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][2 * i + 1]), scale2, neg_base));
+          rs0 += p0;
+          rs1 += p1;
+          pk[c][i] = pack_bf16x2(p0, p1);
+        }
+      l = alpha * l + (rs0 + rs1);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_st16(t_s + 16 * c, pk[c]);
+      const bool rescale = (cnt > 0) && (m_new != m_ref);
+      if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_o + 32 * c, o);
+          tmem_ld_wait();
+          reg_fence(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(t_o + 32 * c, o);
+        }
+      }
+      m_ref = m_new;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bar_pf[w]);
+      ++cnt;
+    }
+    // ---------------------------------------------------------------- epilogue: O / l, lse
+    if (ok && q0 < N) {
+      if (cnt > 0) {
+        const bool got = mbar_wait(&bar_od[w], (cnt - 1) & 1, abort_flag, SITE_FWD_SM_O);
+        ok = __all_sync(0xffffffffu, got);
+        tc_fence_after();
+      }
+      const float inv = (l > 0.f) ? 1.0f / l : 0.0f;
+      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * N + row) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (cnt > 0 && ok) {
+          tmem_ld32(t_o + 32 * c, o);
+          tmem_ld_wait();
+          reg_fence(o);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        uint32_t h[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          h[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+        if (row < N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+        }
+      }
+      if (row < N)
+        p.lse[static_cast<size_t>(bh) * N + row] =
+            (l > 0.f) ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+}  // namespace fa

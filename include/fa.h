@@ -1,0 +1,128 @@
+/*
+ * fa.h -- C ABI of libfa: exact scaled-dot-product attention on NVIDIA B200 (sm_100a),
+ * forward and backward, computed tile by tile so that the N x N score matrix never reaches HBM.
+ *
+ * The operation ("Attention optimisation: FlashAttention and sparse attention", mdooai Ch.04,
+ * sections "core formula" and "formula key points", and its sparse-masking paragraph):
+ *     S_ij = scale * q_i . k_j            (scale is 1/sqrt(d) in the usual setting)
+ *     S_ij = -inf for keys j outside the allowed set of row i
+ *     A    = softmax of each row of S     (each row of A sums to 1)
+ *     O    = A V
+ * computed exactly -- not an approximation -- with the IO-aware tiling of "FlashAttention:
+ * Fast and Memory-Efficient Exact Attention with IO-Awareness" (ai-paper-library summary of
+ * arXiv 2205.14135): tiles of Q, K, V are staged on chip, partial softmax statistics are kept
+ * on chip, and only O and the per-row log-sum-exp go back to HBM.  The backward pass
+ * recomputes the scores from Q, K, V and that log-sum-exp.
+ *
+ * Conventions shared by every entry point
+ *   Layout     q, k, v, o, dO, dq, dk, dv are contiguous [B][H][N][d] row-major (d innermost);
+ *              lse is [B][H][N]. One (b, h) pair is one independent attention problem.
+ *   Masks      the allowed set of row i is the AND of
+ *                causal != 0        : j <= i (square self-attention, lower triangle);
+ *                kv_len != NULL     : j < kv_len[b] (key padding; device int32 [B]);
+ *                block_mask != NULL : block_mask[i/128][j/128] != 0 (device uint8
+ *                                     [ceil(N/128)][ceil(N/128)], shared by every (b, h)).
+ *              A row with no allowed key gets O = 0, lse = -inf and no gradient.
+ *   lse        natural-log log-sum-exp of the scaled, masked logits of the row.
+ *   Memory     every pointer is device memory owned by the caller; the library allocates
+ *              nothing and keeps no pointer after the call returns.
+ *   Execution  asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream); the
+ *              host never waits, so results are ready once the stream reaches this point.
+ *   Errors     a negative fa_status is returned without launching anything when an argument
+ *              is rejected; fa_get_last_error() then describes it.  A CUDA launch failure
+ *              returns FA_ERR_CUDA.  Device-side waits are bounded: a wait that gives up
+ *              records a code that fa_device_status() reports (FA_ERR_TIMEOUT).
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { FA_BF16 = 0, FA_F32 = 1 } fa_dtype;
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID = -1,     /* null pointer, non-positive size, bad scale, unknown dtype   */
+  FA_ERR_UNSUPPORTED = -2, /* head dimension or dtype this build has no kernel for        */
+  FA_ERR_ALIGN = -3,       /* a tensor pointer is not 16-byte aligned (TMA requirement)   */
+  FA_ERR_CUDA = -4,        /* a CUDA call or kernel launch failed                         */
+  FA_ERR_TIMEOUT = -5,     /* a device-side bounded wait gave up (see fa_device_status)  */
+  FA_ERR_WORKSPACE = -6    /* workspace missing, misaligned or smaller than required      */
+} fa_status;
+
+/*
+ * fa_fwd -- forward pass: O = softmax(scale * Q K^T, masked) V and lse.
+ *   dtype FA_BF16: q, k, v, o are bf16, d in {64, 128}; tensor-core (tcgen05) kernel with
+ *                  TMA-fed tiles and an online softmax; fp32 accumulation.
+ *   dtype FA_F32 : q, k, v, o are fp32, 1 <= d <= 128; CUDA-core fp32 kernel.
+ *   scale must be finite and > 0.  N >= 1, B >= 1, H >= 1.
+ *   Pointers q, k, v, o, lse must be 16-byte aligned.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+           int N, int d, float scale, int causal, const uint8_t* block_mask,
+           const int32_t* kv_len, int dtype, void* stream);
+
+/* Bytes of device workspace fa_bwd needs: log2-scaled lse and Dvec ([B][H][ceil128(N)] fp32
+ * each) and the fp32 dQ accumulator ([B][H][N][d]). */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * fa_bwd -- backward pass of fa_fwd from (q, k, v, o, lse, dO), recomputing the scores:
+ *   dV = A^T dO,  dS = A o (dO V^T - rowsum(dO o O)),  dQ = scale dS K,  dK = scale dS^T Q.
+ *   Only FA_BF16 with d in {64, 128}.  o and lse must be fa_fwd's outputs for the same
+ *   arguments.  workspace: device memory of at least fa_bwd_workspace_size() bytes, 256-byte
+ *   aligned, owned by the caller, scratch only (its contents on entry do not matter).
+ *   dq accumulates across key tiles with fp32 atomics, so its last bits may differ between
+ *   runs; dk and dv are deterministic.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+           float scale, int causal, const uint8_t* block_mask, const int32_t* kv_len,
+           int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_fwd_tile_reference -- bf16 forward on CUDA cores for the tile-size numeric-deviation
+ * study of "Is Flash Attention Stable?" (aibr.jp summary, sections 3-4): the running maximum
+ * and sum are rescaled after every tile of `bc` keys (bc in {32, 64, ..., 256}) and P is
+ * rounded to bf16 before P.V, as in a tensor-core kernel with that key-tile width.  Same
+ * layouts, masks and errors as fa_fwd (bf16, 1 <= d <= 128).  Not a fast path.
+ */
+int fa_fwd_tile_reference(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int H, int N, int d, float scale, int causal,
+                          const uint8_t* block_mask, const int32_t* kv_len, int bc,
+                          void* stream);
+
+/* Bytes of workspace fa_naive_fwd needs: the materialised S / P matrix, [B][H][N][N] bf16. */
+size_t fa_naive_workspace_size(int B, int H, int N);
+
+/*
+ * fa_naive_fwd -- the materialised "Baseline Attention" of "Is Flash Attention Stable?":
+ * S = bf16(scale Q K^T) written to the workspace, row softmax in fp32 read from it with
+ * P = bf16 written back, then O = bf16(P V) with fp32 accumulation.  bf16, 1 <= d <= 128.
+ * A deviation and speed reference, not a fast path.
+ */
+int fa_naive_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, float scale, int causal, const uint8_t* block_mask,
+                 const int32_t* kv_len, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Message for the most recent non-OK status returned on this host thread. */
+const char* fa_get_last_error(void);
+
+/*
+ * fa_device_status -- synchronises the current device, then returns FA_OK, or FA_ERR_TIMEOUT
+ * if a kernel's bounded wait gave up since the last call (the first such event's code,
+ * (site << 16) | (block index & 0xffff), is stored in *code when code != NULL), and clears it.
+ * Returns FA_ERR_CUDA if the synchronisation itself reports an error.
+ */
+int fa_device_status(unsigned int* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

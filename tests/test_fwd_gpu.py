@@ -1,0 +1,140 @@
+"""Forward parity on the GPU: the CUDA path (through the C ABI) against the FP64 oracle on the
+same seeded inputs.  Small cases span several tiles and ragged tails and are compared element
+by element; the full-size workloads are compared in full where the oracle is quick, else on
+sampled rows, in the launch configuration the bench times."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic as syn
+from gpu_util import (compare_lse, compare_o, f64, oracle_fwd, to_gpu)
+
+pytestmark = pytest.mark.gpu
+
+
+def run_fwd(fa, g):
+    o, lse = fa.fwd(g["q"], g["k"], g["v"], g["scale"], g["causal"], g["block_mask"], g["kv_len"])
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    return o, lse
+
+
+SMALL = [
+    # B, H, N, d, causal, kv_len, block-mask kind
+    (2, 3, 700, 64, False, None, None),
+    (2, 3, 700, 64, True, None, None),
+    (1, 2, 1000, 128, True, None, None),
+    (1, 2, 777, 128, False, None, None),
+    (3, 2, 512, 64, False, [130, 512, 301], None),
+    (2, 2, 640, 128, True, [640, 333], None),
+    (1, 3, 900, 64, False, None, "band"),
+    (1, 2, 1100, 128, True, None, "band"),
+    (1, 1, 1, 64, False, None, None),
+    (1, 1, 8, 128, True, None, None),
+    (1, 2, 129, 64, True, None, None),
+    (2, 1, 300, 64, False, [1, 300], None),
+]
+
+
+def _bm(kind, N):
+    if kind is None:
+        return None
+    return syn.block_mask_band_global(N)
+
+
+@pytest.mark.parametrize("case", range(len(SMALL)))
+def test_fwd_small_elementwise(cuda_lib, case):
+    B, H, N, d, causal, L, bmk = SMALL[case]
+    x = syn.make_inputs(B, H, N, d, "bf16", seed=500 + case, causal=causal,
+                        kv_len=None if L is None else np.array(L, np.int32),
+                        block_mask=_bm(bmk, N), with_grad=False)
+    o, lse = run_fwd(cuda_lib, to_gpu(x))
+    o_ref, lse_ref = oracle_fwd(x)
+    compare_o(f64(o), o_ref)
+    compare_lse(f64(lse), lse_ref)
+
+
+def test_fwd_fully_masked_rows(cuda_lib):
+    """Query block 1 keeps no key block: its rows give O = 0 and lse = -inf."""
+    N = 384
+    bm = np.ones((3, 3), np.uint8)
+    bm[1, :] = 0
+    x = syn.make_inputs(1, 2, N, 64, "bf16", seed=77, block_mask=bm, with_grad=False)
+    o, lse = run_fwd(cuda_lib, to_gpu(x))
+    o_ref, lse_ref = oracle_fwd(x)
+    assert torch.all(o[:, :, 128:256] == 0)
+    assert torch.all(torch.isneginf(lse[:, :, 128:256]))
+    compare_o(f64(o), o_ref)
+    compare_lse(f64(lse), lse_ref)
+
+
+def test_fwd_fp32_single_head(cuda_lib):
+    """fp32 workload, B1 H1 N128 d64: every element within 1e-5 of the oracle."""
+    x = syn.workload_inputs("fp32_single_head")
+    o, lse = run_fwd(cuda_lib, to_gpu(x))
+    o_ref, lse_ref = oracle_fwd(x)
+    compare_o(f64(o), o_ref, "f32")
+    compare_lse(f64(lse), lse_ref, 1e-5)
+
+
+@pytest.mark.parametrize("N,d,causal", [(300, 100, True), (257, 7, False)])
+def test_fwd_fp32_odd_shapes(cuda_lib, N, d, causal):
+    x = syn.make_inputs(1, 2, N, d, "f32", seed=31, causal=causal, with_grad=False)
+    o, lse = run_fwd(cuda_lib, to_gpu(x))
+    o_ref, lse_ref = oracle_fwd(x)
+    compare_o(f64(o), o_ref, "f32")
+    compare_lse(f64(lse), lse_ref, 1e-5)
+
+
+@pytest.mark.parametrize("name", ["gpt2_causal", "bert_padding"])
+def test_fwd_workload_full(cuda_lib, name):
+    x = syn.workload_inputs(name, with_grad=False)
+    o, lse = run_fwd(cuda_lib, to_gpu(x))
+    o_ref, lse_ref = oracle_fwd(x)
+    compare_o(f64(o), o_ref)
+    compare_lse(f64(lse), lse_ref)
+
+
+@pytest.mark.parametrize("name", ["long_causal", "block_sparse"])
+def test_fwd_workload_sampled_rows(cuda_lib, name):
+    """Full-size launch; the oracle computes 768 sampled rows one by one."""
+    x = syn.workload_inputs(name, with_grad=False)
+    o, lse = run_fwd(cuda_lib, to_gpu(x))
+    B, H, N, d = x["B"], x["q"].shape[1], x["N"], x["d"]
+    rng = np.random.default_rng(4242)
+    rows = rng.choice(B * H * N, size=700, replace=False)
+    edge = np.array([0, 127, 128, 255, 256, N - 1, N - 128, B * H * N - 1])
+    rows = np.unique(np.concatenate([rows, edge]))
+    o_ref, lse_ref = oracle.attn_fwd_rows(x["q"], x["k"], x["v"], x["scale"], rows, x["causal"],
+                                          x["block_mask"], x["kv_len"])
+    o_g = f64(o).reshape(-1, d)[rows]
+    l_g = f64(lse).reshape(-1)[rows]
+    compare_o(o_g, o_ref)
+    compare_lse(l_g, lse_ref)
+    # every output is finite and the row-sum invariant holds in aggregate: |O| <= max |V|
+    assert torch.isfinite(o.float()).all()
+    assert o.float().abs().max().item() <= x["v"].float().abs().max().item() + 1e-2
+
+
+def test_fwd_deterministic(cuda_lib):
+    x = to_gpu(syn.make_inputs(2, 2, 600, 128, "bf16", seed=9, causal=True, with_grad=False))
+    o1, l1 = run_fwd(cuda_lib, x)
+    o2, l2 = run_fwd(cuda_lib, x)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_tile_reference_and_naive_within_tolerance(cuda_lib):
+    """The deviation-study kernels compute the same attention (bf16 tolerance)."""
+    x = syn.make_inputs(2, 2, 520, 64, "bf16", seed=12, causal=True, with_grad=False)
+    g = to_gpu(x)
+    o_ref, lse_ref = oracle_fwd(x)
+    for bc in (64, 128, 256):
+        o, lse = cuda_lib.fwd_tile_reference(g["q"], g["k"], g["v"], bc, g["scale"], True)
+        torch.cuda.synchronize()
+        compare_o(f64(o), o_ref)
+        compare_lse(f64(lse), lse_ref)
+    o, lse = cuda_lib.naive_fwd(g["q"], g["k"], g["v"], g["scale"], True)
+    torch.cuda.synchronize()
+    compare_o(f64(o), o_ref)
+    compare_lse(f64(lse), lse_ref, 2e-2)
