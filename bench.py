@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Throughput of exact tiled attention (forward + backward) on B200, one JSON line.
+
+A step is one pass of the whole path over one batch: fa_fwd (O, lse) then fa_bwd (dQ, dK, dV)
+on the long-context causal workload (B1 H16 N16384 d128, Q,K ~ 2 N(0,1), bf16), inputs
+resident in HBM.  FLOPs count only unmasked (i, j) pairs P: 4 d P forward, 10 d P backward.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun) every rank runs its own replica of the workload (the (b, h) problems
+are independent, so there is no data-path collective; scaling is weak) and the time is the
+max over ranks.  ``--impl reference`` times the FP64 CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic as syn  # noqa: E402
+
+WORKLOAD = "long_causal"
+METRIC = "attention fwd/bwd TFLOP/s on 1 B200 and % of BF16 tensor peak; max err vs FP64"
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=16384,
+                    help="query rows in the oracle's timed sample")
+    ap.add_argument("--ref-rows", type=int, default=1024,
+                    help="query rows per step of the reference (oracle) arm")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- accounting
+def flops(x: dict, H: int) -> tuple[float, float]:
+    kv = None if x["kv_len"] is None else x["kv_len"].numpy()
+    bm = None if x["block_mask"] is None else x["block_mask"].numpy()
+    P = float(syn.allowed_pairs(x["N"], x["causal"], kv, x["B"], bm).sum()) * H
+    return 4.0 * x["d"] * P, 10.0 * x["d"] * P
+
+
+def row_pairs(x: dict, rows: np.ndarray) -> np.ndarray:
+    """Unmasked keys of each flat row (counting only; used for the oracle sample's FLOPs)."""
+    N, H = x["N"], x["q"].shape[1]
+    i = rows % N
+    b = rows // N // H
+    L = np.full(len(rows), N) if x["kv_len"] is None else x["kv_len"].numpy()[b]
+    n = np.minimum(i + 1, L) if x["causal"] else L.copy()
+    if x["block_mask"] is not None:
+        bm = x["block_mask"].numpy()
+        n = np.array([sum(max(0, min((J + 1) * 128, Lr, (ir + 1) if x["causal"] else Lr) - J * 128)
+                          for J in range(bm.shape[1]) if bm[ir // 128, J])
+                      for ir, Lr in zip(i, L)])
+    return n.astype(np.float64)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def csrc_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "exact_io_aware_98_b200", "csrc")
+    for name in sorted(os.listdir(d)):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    e = t.get(kernel, {})
+    if e.get("workload") != workload or e.get("csrc_hash") != csrc_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.ok = False
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as exc:  # no NVML: report the absence, never guess
+            self.err = repr(exc)
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if bits & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self) -> dict:
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        self._stop.set()
+        self._t.join()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank: int, world: int, dist):
+    import exact_io_aware_98_b200 as fa
+    fa.load()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    x = syn.workload_inputs(args.workload)
+    H = x["q"].shape[1]
+    B, N, d = x["B"], x["N"], x["d"]
+    g = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in x.items()}
+    f_fwd, f_bwd = flops(x, H)
+    o = torch.empty_like(g["q"])
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty_like(g["q"]) for _ in range(3))
+    ws = torch.empty(fa.bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    kw = dict(scale=g["scale"], causal=g["causal"], block_mask=g["block_mask"],
+              kv_len=g["kv_len"])
+
+    def step():
+        fa.fwd(g["q"], g["k"], g["v"], out=o, lse=lse, **kw)
+        fa.bwd(g["q"], g["k"], g["v"], o, lse, g["do"], workspace=ws, dq=dq, dk=dk, dv=dv, **kw)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if fa.device_status() != 0:
+        raise RuntimeError("a device-side wait gave up during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler = ClockSampler(dev.index)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    for s in range(K):
+        ev[s][0].record()
+        fa.fwd(g["q"], g["k"], g["v"], out=o, lse=lse, **kw)
+        ev[s][1].record()
+        fa.bwd(g["q"], g["k"], g["v"], o, lse, g["do"], workspace=ws, dq=dq, dk=dk, dv=dv, **kw)
+        ev[s][2].record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if dist is not None:
+        dist.barrier()
+    total_ms = ev[0][0].elapsed_time(ev[K - 1][2])
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    t = torch.tensor([total_ms, fwd_ms, bwd_ms], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, fwd_ms, bwd_ms = (float(v) for v in t.tolist())
+    status = fa.device_status()
+
+    # ---- end to end through the public API: pinned host inputs in, results back to host
+    e2e = None
+    if not args.no_e2e:
+        hin = {k: x[k].pin_memory() for k in ("q", "k", "v", "do")}
+        hout = {"o": torch.empty_like(hin["q"]).pin_memory(),
+                "lse": torch.empty((B, H, N), dtype=torch.float32).pin_memory(),
+                "dq": torch.empty_like(hin["q"]).pin_memory(),
+                "dk": torch.empty_like(hin["q"]).pin_memory(),
+                "dv": torch.empty_like(hin["q"]).pin_memory()}
+        din = {k: torch.empty_like(g[k]) for k in hin}
+        h2d = sum(t.numel() * t.element_size() for t in hin.values())
+        d2h = sum(t.numel() * t.element_size() for t in hout.values())
+
+        def e2e_step():
+            for k in hin:
+                din[k].copy_(hin[k], non_blocking=True)
+            fa.fwd(din["q"], din["k"], din["v"], out=o, lse=lse, **kw)
+            fa.bwd(din["q"], din["k"], din["v"], o, lse, din["do"], workspace=ws, dq=dq, dk=dk,
+                   dv=dv, **kw)
+            for k, src in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+                hout[k].copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        Ke = max(3, min(K, 10))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(Ke):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if dist is not None:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        ms_e = float(te.item()) / Ke
+        e2e = {"value": round((f_fwd + f_bwd) * world / (ms_e * 1e-3) / 1e12, 3),
+               "unit": "TFLOP/s", "ms_per_step": round(ms_e, 4), "steps": Ke,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    ms_step = total_ms / K
+    value = (f_fwd + f_bwd) * world / (ms_step * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    fwd_tf = f_fwd / (fwd_ms * 1e-3) / 1e12
+    bwd_tf = f_bwd / (bwd_ms * 1e-3) / 1e12
+    dom = (("fa_bwd_sm100_kernel", bwd_tf, f_bwd) if bwd_ms >= fwd_ms
+           else ("fa_fwd_sm100_kernel", fwd_tf, f_fwd))
+    roof = {"bound": "tensor", "kernel": dom[0], "achieved": round(dom[1], 2),
+            "peak": sustained, "unit": "TFLOP/s", "frac": round(dom[1] / sustained, 4),
+            "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+            "frac_of_burst": round(dom[1] / burst, 4),
+            "frac_of_nominal_2250": round(dom[1] / NOMINAL_BF16_TFLOPS, 4),
+            "flop_per_launch": dom[2], "traffic": traffic_for(dom[0], args.workload),
+            "note": "achieved = algorithmic FLOP / CUDA-event duration of the whole fa_bwd call "
+                    "(preprocess + tensor-core main kernel + dQ convert) or of fa_fwd (one "
+                    "launch); traffic = ncu DRAM bytes of the main kernel's launch"}
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1); Q,K x2), no dataset",
+        "config": {"workload": f"{args.workload}: {syn.WORKLOADS[args.workload].description}",
+                   "B": B, "H": H, "N": N, "d": d,
+                   "mask": syn.WORKLOADS[args.workload].mask,
+                   "step": "fa_fwd + fa_bwd", "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: Q,K,V,dO are 4 x %.0f MiB per step"
+                         % (x["q"].numel() * 2 / 2**20)},
+        "fwd": {"ms": round(fwd_ms, 4), "tflops": round(fwd_tf, 2),
+                "frac_sustained": round(fwd_tf / sustained, 4)},
+        "bwd": {"ms": round(bwd_ms, 4), "tflops": round(bwd_tf, 2),
+                "frac_sustained": round(bwd_tf / sustained, 4)},
+        "roofline": roof,
+        "clocks": clocks,
+        "gpu_launches": K * 4,
+        "device_status": status,
+        "e2e": e2e,
+    }
+    return line, (x, g, o, lse, dq)
+
+
+# ----------------------------------------------------------------------------- CPU baseline leg
+def cpu_baseline_leg(args, x, o, lse, dq):
+    """Times the FP64 oracle on a bounded row sample of the same workload on this host's cores
+    and, from the same oracle results, reports the GPU outputs' error on those rows."""
+    import oracle
+    N, H, d = x["N"], x["q"].shape[1], x["d"]
+    xd = {k: x[k].double().numpy() for k in ("q", "k", "v", "do")}  # widened once, untimed
+    rng = np.random.default_rng(1234)
+    rows = np.sort(rng.choice(x["B"] * H * N, size=min(args.cpu_rows, x["B"] * H * N),
+                              replace=False))
+    t0 = time.perf_counter()
+    o_ref, l_ref = oracle.attn_fwd_rows(xd["q"], xd["k"], xd["v"], x["scale"], rows,
+                                        x["causal"], x["block_mask"], x["kv_len"])
+    dq_ref = oracle.attn_bwd_dq_rows(xd["q"], xd["k"], xd["v"], xd["do"], x["scale"], rows,
+                                     x["causal"], x["block_mask"], x["kv_len"])
+    dt = time.perf_counter() - t0
+    n = row_pairs(x, rows)
+    fl = 10.0 * d * n.sum()   # forward 4 d n_i + recompute S, dP and dQ 6 d n_i
+    o_g = o.float().cpu().double().numpy().reshape(-1, d)[rows]
+    l_g = lse.float().cpu().double().numpy().reshape(-1)[rows]
+    dq_g = dq.float().cpu().double().numpy().reshape(-1, d)[rows]
+    eo = np.abs(o_g - o_ref)
+    fin = np.isfinite(l_ref)
+    el = np.abs(l_g[fin] - l_ref[fin]) if fin.any() else np.zeros(1)
+    edq = np.abs(dq_g - dq_ref) / max(np.abs(dq_ref).max(), 1e-30)
+    cpu = {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+           "kind": "oracle",
+           "sample": f"O, lse and dQ of {len(rows)} random query rows of {args.workload} "
+                     f"(FP64, S and A rows materialised); {dt:.1f} s wall",
+           "seconds": round(dt, 2)}
+    err = {"rows": len(rows), "o_max": float(eo.max()), "o_mean": float(eo.mean()),
+           "lse_max": float(el.max()), "dq_max_rel": float(edq.max()),
+           "dq_mean_rel": float(edq.mean()),
+           "tolerance": "O: max 2e-2, mean 2e-3; dQ: same relative to max|ref|"}
+    return cpu, err
+
+
+def deviation_sweep():
+    """Numeric deviation vs the FP64 golden across key-tile widths, next to the naive kernel
+    (the microbenchmark of "Is Flash Attention Stable?"), on 32 heads of the padding workload."""
+    import oracle
+    import exact_io_aware_98_b200 as fa
+    x = syn.workload_inputs("bert_padding", with_grad=False, H=2)
+    g = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
+    gold, _ = oracle.attn_fwd(x["q"], x["k"], x["v"], x["scale"], False, None, x["kv_len"])
+    out = {}
+
+    def stat(t):
+        e = np.abs(t.float().cpu().double().numpy() - gold)
+        return {"max": float(e.max()), "mean": float(e.mean())}
+    kw = dict(scale=g["scale"], kv_len=g["kv_len"])
+    o_tc, _ = fa.fwd(g["q"], g["k"], g["v"], **kw)
+    out["tcgen05_Br128_Bc128_lazy"] = stat(o_tc)
+    for bc in (64, 128, 256):
+        o_t, _ = fa.fwd_tile_reference(g["q"], g["k"], g["v"], bc, **kw)
+        out[f"tile_Bc{bc}"] = stat(o_t)
+    o_n, _ = fa.naive_fwd(g["q"], g["k"], g["v"], **kw)
+    out["naive_materialised"] = stat(o_n)
+    diff = (o_tc.float() - o_n.float()).abs()
+    out["tcgen05_vs_naive"] = {"max": float(diff.max()), "mean": float(diff.mean())}
+    out["note"] = ("row-wise arithmetic does not depend on Br (query-tile height), so the sweep "
+                   "varies Bc; the tcgen05 kernel is Br=Bc=128 with a lazy (2^8) rescale")
+    return out
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, world: int):
+    import oracle
+    x = syn.workload_inputs(args.workload)
+    N, H, d = x["N"], x["q"].shape[1], x["d"]
+    xd = {k: x[k].double().numpy() for k in ("q", "k", "v", "do")}  # widened once, untimed
+    rng = np.random.default_rng(99)
+    R = min(args.ref_rows, x["B"] * H * N)
+
+    def one(seed):
+        rows = np.sort(np.random.default_rng(seed).choice(x["B"] * H * N, size=R, replace=False))
+        t0 = time.perf_counter()
+        oracle.attn_fwd_rows(xd["q"], xd["k"], xd["v"], x["scale"], rows, x["causal"],
+                             x["block_mask"], x["kv_len"])
+        oracle.attn_bwd_dq_rows(xd["q"], xd["k"], xd["v"], xd["do"], x["scale"], rows,
+                                x["causal"], x["block_mask"], x["kv_len"])
+        return time.perf_counter() - t0, 10.0 * d * row_pairs(x, rows).sum()
+
+    for w in range(args.warmup):
+        one(int(rng.integers(1 << 30)))
+    tt, ff = 0.0, 0.0
+    for s in range(args.steps):
+        dt, fl = one(int(rng.integers(1 << 30)))
+        tt += dt
+        ff += fl
+    value = ff / tt / 1e12
+    sample = f"O, lse and dQ of {R} random query rows of {args.workload} per step (FP64)"
+    return {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(tt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{args.workload}: {syn.WORKLOADS[args.workload].description}",
+                       "B": x["B"], "H": H, "N": N, "d": d, "parallelism": "host cores"},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
+                             "cores": oracle.num_threads(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, world)), flush=True)
+        return
+    dist = None
+    if world > 1:
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        line, (x, g, o, lse, dq) = run_ours(args, rank, world, dist)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            cpu, err = cpu_baseline_leg(args, x, o, lse, dq)
+            line["cpu_baseline"] = cpu
+            line["max_err_vs_fp64"] = err
+            line["deviation_sweep"] = deviation_sweep()
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

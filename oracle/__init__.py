@@ -72,6 +72,11 @@ def _load():
         lib.oracle_softmax_av.restype = None
         lib.oracle_softmax_av.argtypes = [_dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           _dp, _dp, _dp]
+        lib.oracle_attn_bwd_dq_rows.restype = ctypes.c_int
+        lib.oracle_attn_bwd_dq_rows.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                                ctypes.c_int, _u8p, ctypes.c_int, _i32p, _i64p,
+                                                ctypes.c_int, _dp]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -154,6 +159,24 @@ def attn_bwd(q, k, v, do, scale: float, causal: bool = False, block_mask=None, k
     if rc != 0:
         raise RuntimeError(f"oracle_attn_bwd failed ({rc})")
     return dq, dk, dv
+
+
+def attn_bwd_dq_rows(q, k, v, do, scale: float, rows: Sequence[int], causal: bool = False,
+                     block_mask=None, kv_len=None, block: int = 128):
+    """dQ of selected rows (flat (b*H + h)*N + i), float64 [len(rows), d]."""
+    lib = _load()
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, H, N, d = q.shape
+    bm, kl = _masks(block_mask, kv_len)
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    dq = np.zeros((len(r), d), np.float64)
+    rc = lib.oracle_attn_bwd_dq_rows(_ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), _ptr(do, _dp),
+                                     B, H, N, d, float(scale), int(bool(causal)),
+                                     _ptr(bm, _u8p), block, _ptr(kl, _i32p), _ptr(r, _i64p),
+                                     len(r), _ptr(dq, _dp))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_bwd_dq_rows failed ({rc})")
+    return dq
 
 
 def attn_probs(q, k, scale: float, causal: bool = False, block_mask=None, kv_len_b: int = -1,

@@ -306,3 +306,51 @@ int oracle_attn_bwd(const double *q, const double *k, const double *v, const dou
     free(dS);
     return 0;
 }
+
+/* dQ of selected query rows only (flat index (b*H + h)*N + i): the backward's definition
+ * restricted to those rows -- dQ_i needs only row i of A and of dA. */
+int oracle_attn_bwd_dq_rows(const double *q, const double *k, const double *v, const double *dO,
+                            int B, int H, int N, int d, double scale, int causal,
+                            const uint8_t *block_mask, int block, const int32_t *kv_len,
+                            const int64_t *rows, int nrows, double *dq_rows)
+{
+    int bad = 0;
+    #pragma omp parallel
+    {
+        double *a = (double *)malloc(sizeof(double) * (size_t)N);
+        double *ds = (double *)malloc(sizeof(double) * (size_t)N);
+        #pragma omp for schedule(dynamic, 1)
+        for (int r = 0; r < nrows; ++r) {
+            int64_t flat = rows[r];
+            int64_t bh = flat / N;
+            int i = (int)(flat % N);
+            int b = (int)(bh / H);
+            if (flat < 0 || b >= B) { bad = 1; continue; }
+            mask_t m = make_mask(N, causal, block_mask, block, kv_len, b);
+            size_t off = (size_t)bh * (size_t)N * d;
+            const double *kh = k + off, *vh = v + off, *dOi = dO + off + (size_t)i * d;
+            logits_row(q + off + (size_t)i * d, kh, N, d, scale, &m, i, a);
+            softmax_row(a, N);
+            double delta = 0.0;
+            for (int j = 0; j < N; ++j) {
+                double dot = 0.0;
+                const double *vj = vh + (size_t)j * d;
+                for (int c = 0; c < d; ++c) dot += dOi[c] * vj[c];
+                ds[j] = dot;                               /* dA_ij */
+                delta += a[j] * dot;
+            }
+            double *out = dq_rows + (size_t)r * d;
+            for (int c = 0; c < d; ++c) out[c] = 0.0;
+            for (int j = 0; j < N; ++j) {
+                double w = a[j] * (ds[j] - delta);        /* dS_ij */
+                if (w == 0.0) continue;
+                const double *kj = kh + (size_t)j * d;
+                for (int c = 0; c < d; ++c) out[c] += w * kj[c];
+            }
+            for (int c = 0; c < d; ++c) out[c] *= scale;
+        }
+        free(a);
+        free(ds);
+    }
+    return bad ? -1 : 0;
+}

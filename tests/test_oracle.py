@@ -292,3 +292,20 @@ def test_backward_head_subset():
     for a, b in zip(full, part):
         assert np.array_equal(a[0, 2], b[0, 2])
         assert np.all(b[0, :2] == 0.0)
+
+
+@pytest.mark.parametrize("case", range(len(CASES)))
+def test_dq_rows_match_brute_force(case):
+    """The row-restricted dQ equals the brute-force chain rule on the same rows."""
+    N, d, causal, L, bml, block = CASES[case]
+    q, k, v, do = _case(N, d, causal, L, bml, block, 300 + case)
+    scale = 0.4
+    bm = None if bml is None else np.array(bml, np.uint8)
+    gq, _, _ = bf.backward_head(q.tolist(), k.tolist(), v.tolist(), do.tolist(), scale, causal,
+                                bml, block, L)
+    rows = list(range(N))[::-1]
+    dq = oracle.attn_bwd_dq_rows(q[None, None], k[None, None], v[None, None], do[None, None],
+                                 scale, rows, causal, bm,
+                                 None if L is None else np.array([L], np.int32), block)
+    ref = np.array(gq)[rows]
+    assert np.max(np.abs(dq - ref)) < 1e-12 * max(1.0, np.max(np.abs(ref)))
