@@ -28,6 +28,8 @@ SIGNATURES = {
     "fa_bwd_workspace_size": (_sz, [_i, _i, _i, _i]),
     "fa_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp,
                     _vp, _i, _vp, _sz, _vp]),
+    "fa_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
+                            _vp, _vp, _i, _vp]),
     "fa_fwd_tile_reference": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp,
                                    _i, _vp]),
     "fa_naive_workspace_size": (_sz, [_i, _i, _i]),
@@ -148,6 +150,27 @@ def bwd(q, k, v, o, lse, do, scale: Optional[float] = None, causal: bool = False
                     _ptr(dv), B, H, N, d, s, int(causal), bm, kl, _dtype_code(q), _ptr(ws),
                     ws.numel(), _stream())
     _check(rc, "fa_bwd")
+    return dq, dk, dv
+
+
+def bwd_noalloc(q, k, v, o, lse, do, scale: Optional[float] = None, causal: bool = False,
+                block_mask=None, kv_len=None, dq=None, dk=None, dv=None):
+    """fa_bwd without a workspace: for callers that cannot allocate device memory.  The
+    library's own fixed 32 MiB scratch is used instead; calls on one device must not overlap."""
+    lib = load()
+    B, H, N, d = q.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _require(t, n, q.dtype)
+    _require(lse, "lse", torch.float32)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    bm, kl = _masks(block_mask, kv_len)
+    s = default_scale(d) if scale is None else float(scale)
+    rc = lib.fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq),
+                            _ptr(dk), _ptr(dv), B, H, N, d, s, int(causal), bm, kl,
+                            _dtype_code(q), _stream())
+    _check(rc, "fa_bwd_noalloc")
     return dq, dk, dv
 
 

@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "fa.h"
 #include "fa_bwd_sm100.cuh"
@@ -309,3 +310,91 @@ int fa_naive_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// Backward pass without any caller-provided or library-allocated workspace.
+//
+// Some callers cannot hand the library a device buffer: they run inside a host framework that
+// owns every device allocation (a plugin interface that passes in only the input and output
+// tensors, a fixed-budget memory pool), or they must not call cudaMalloc / cudaFree because
+// those calls can synchronise the whole device.  fa_bwd_noalloc serves them: its scratch (the
+// log2-scaled lse, Dvec and the fp32 dQ accumulator) lives in the fixed-size array below, which
+// the CUDA driver places on every device that loads this library and keeps there until the
+// process exits.  Nothing is allocated per call.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(32) << 20;  // 32 MiB per device
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device.  The host-side name of the array
+// is only a stand-in, never a device address, so the address is looked up once per device (with
+// that device current) and cached.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(FA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(FA_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                              const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                              int B, int H, int N, int d, float scale, int causal,
+                              const uint8_t* block_mask, const int32_t* kv_len, int dtype,
+                              void* stream) {
+  int rc = common_checks(q, k, v, o, lse, B, H, N, d, scale);
+  if (rc != FA_OK) return rc;
+  if (!dO || !dq || !dk || !dv) return fail(FA_ERR_INVALID, "null gradient pointer");
+  if (!aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return fail(FA_ERR_ALIGN, "gradient pointers must be 16-byte aligned");
+  if (dtype != FA_BF16) {
+    if (dtype == FA_F32) return fail(FA_ERR_UNSUPPORTED, "fp32 backward is not built");
+    return fail(FA_ERR_INVALID, "unknown dtype %d", dtype);
+  }
+  if (d != 64 && d != 128)
+    return fail(FA_ERR_UNSUPPORTED, "bf16 backward supports d in {64, 128}, got %d", d);
+  const BwdWs ws = bwd_ws(B, H, N, d);
+  if (ws.total > kNoAllocScratchBytes)
+    return fail(FA_ERR_WORKSPACE,
+                "fa_bwd_noalloc: this problem needs %zu bytes of scratch but the built-in "
+                "scratch holds %zu; use fa_bwd with a caller-provided workspace",
+                ws.total, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch)) != FA_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(scratch);
+  const int BH = B * H;
+  // The preprocess kernel rewrites lse2 / Dvec and zeroes the dQ accumulator, so whatever the
+  // previous call left in the scratch never leaks into this one.
+  const long long pre_rows = static_cast<long long>(BH) * ws.n_pad;
+  fa::bwd_preprocess_kernel<<<static_cast<unsigned>((pre_rows + 7) / 8), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse,
+      reinterpret_cast<float*>(wsb + ws.lse2), reinterpret_cast<float*>(wsb + ws.dvec),
+      reinterpret_cast<float*>(wsb + ws.dq), BH, N, ws.n_pad, d);
+  if ((rc = check_launch("bwd_preprocess_kernel")) != FA_OK) return rc;
+  if (d == 64)
+    rc = launch_bwd<64>(q, k, v, dO, dk, dv, B, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+  else
+    rc = launch_bwd<128>(q, k, v, dO, dk, dv, B, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+  if (rc != FA_OK) return rc;
+  const long long n = static_cast<long long>(BH) * N * d;
+  fa::dq_convert_kernel<<<static_cast<unsigned>((n / 8 + 255) / 256 + 1), 256, 0, s>>>(
+      reinterpret_cast<const float*>(wsb + ws.dq), static_cast<__nv_bfloat16*>(dq), n, scale);
+  return check_launch("dq_convert_kernel");
+}

@@ -86,6 +86,29 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            int dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_bwd_noalloc -- the backward pass of fa_bwd for callers that cannot provide or allocate
+ * device memory.  The pages have no counterpart: this entry point exists for integration.
+ *   Who needs it: code running inside a host framework that owns every device allocation (a
+ *   plugin interface that hands over only the input and output tensors, a fixed-budget memory
+ *   pool), or code that must not call cudaMalloc / cudaFree because they can synchronise the
+ *   whole device.  This call allocates nothing: its scratch (log2-scaled lse, Dvec and the fp32
+ *   dQ accumulator, sized as fa_bwd_workspace_size() reports) is a fixed 32 MiB array that the
+ *   library keeps on every device that loads it, until the process exits.
+ *   Arguments, layouts, masks and results are those of fa_bwd, without the workspace pair.
+ *   Limit: problems whose fa_bwd_workspace_size(B, H, N, d) exceeds 32 MiB (33554432 bytes)
+ *   are rejected with FA_ERR_WORKSPACE before anything is launched.
+ *   Set-up: the first call on a device looks up the array's device address (with that device
+ *   current) and caches it; make that first call before any stream capture.
+ *   Sharing: every call on a device uses the same scratch and leaves its contents behind; each
+ *   call re-initialises everything it reads, but two calls that overlap on the GPU (different
+ *   streams, no ordering between them) race on the scratch and give wrong gradients.
+ */
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                   float scale, int causal, const uint8_t* block_mask, const int32_t* kv_len,
+                   int dtype, void* stream);
+
+/*
  * fa_fwd_tile_reference -- bf16 forward on CUDA cores for the tile-size numeric-deviation
  * study of "Is Flash Attention Stable?" (aibr.jp summary, sections 3-4): the running maximum
  * and sum are rescaled after every tile of `bc` keys (bc in {32, 64, ..., 256}) and P is
