@@ -171,7 +171,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void
   p.causal = causal ? 1 : 0;
   const long long grid = static_cast<long long>(p.n_ktiles) * BH;
   if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
-  fa::fa_bwd_sm100_kernel<D><<<static_cast<unsigned>(grid), 320, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
+  fa::fa_bwd_sm100_kernel<D><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
   return check_launch("fa_bwd_sm100_kernel");
 }
 

@@ -15,17 +15,20 @@
 // see them (causal, key padding and block mask skip whole tiles).  Per query tile of BM rows:
 //   S^T  = K Q^T     (M=128 keys, N=BM, K=D)      smem x smem  -> TMEM
 //   dP^T = V dO^T    (M=128, N=BM, K=D)           smem x smem  -> TMEM
-//   compute warpgroup: P^T, dS^T in bf16 back into TMEM (over S^T / dP^T) and dS^T to smem
+//   compute warpgroups (two, each owning half of the BM query columns): P^T and dS^T in bf16
+//   back into TMEM (each over the front half of its own S^T / dP^T columns) and dS^T to smem
 //   dV  += P^T dO    (M=128, N=D, K=BM)           TMEM x smem  -> TMEM
 //   dK  += dS^T Q    (M=128, N=D, K=BM)           TMEM x smem  -> TMEM
 //   D=64 : dQ   = dS K     (M=BM=128, N=64,  K=128) smem x smem -> TMEM (row per lane)
 //   D=128: dQ^T = K^T dS^T (M=128,    N=BM=64, K=128) smem x smem -> TMEM (column per lane)
 //   dQ warpgroup: TMEM -> fp32 red.global.add into the dQ workspace.
-// The MMA thread issues dV(t), S(t+1), dK(t), dP(t+1), dQ(t): in-order execution lets S(t+1)
-// reuse the TMEM that dV(t) read P^T(t) from, and dP(t+1) the TMEM of dS^T(t), so the
-// compute warpgroup works on step t+1 while dQ(t) runs.
+// Hand-offs per step: P ready (-> dV(t), then S(t+1)) and dS ready (-> dK(t), then dP(t+1),
+// then dQ(t)).  In-order MMA execution lets S(t+1) reuse the TMEM that dV(t) read P^T(t) from,
+// and dP(t+1) the TMEM of dS^T(t); the compute warpgroups compute dS(t) while dV(t) and S(t+1)
+// run, and P(t+1) while dK(t), dP(t+1) and dQ(t) run.
 //
-// CTA: 320 threads. warps 0-3 compute, warp 4 TMA producer, warp 5 MMA issuer, warps 6-9 dQ.
+// CTA: 448 threads. warps 0-7 compute (two warpgroups), warp 8 TMA producer, warp 9 MMA
+// issuer, warps 10-13 dQ.
 #pragma once
 #include "ptx.cuh"
 
@@ -49,7 +52,7 @@ template <int D>
 struct BwdLayout {
   static constexpr int BN = 128;                  // keys per CTA
   static constexpr int BM = D == 64 ? 128 : 64;   // query rows per step
-  static constexpr int QST = 2;
+  static constexpr int QST = 3;                   // Q/dO/lse/Dvec stages
   static constexpr int SUB = D / 64;
   static constexpr int KV_SUBTILE = 128 * 128;
   static constexpr int Q_SUBTILE = BM * 128;
@@ -65,8 +68,12 @@ struct BwdLayout {
   static constexpr int OFF_LSE = OFF_DS + 2 * DS_TILE;
   static constexpr int OFF_DVEC = OFF_LSE + QST * BM * 4;
   static constexpr int OFF_BAR = OFF_DVEC + QST * BM * 4;
-  // kv, q_full[QST], q_empty[QST], sdp_full, ds_full, dq_full[2], dq_empty[2], kv_done, fin
-  static constexpr int NBAR = 1 + 2 * QST + 1 + 1 + 2 + 2 + 1 + 1;
+  // kv, q_full[QST], q_empty[QST], s_full, dp_full, p_full, ds_full, dq_full[2], dq_empty[2],
+  // kv_done, fin
+  static constexpr int NBAR = 1 + 2 * QST + 4 + 2 + 2 + 1 + 1;
+  static constexpr int THREADS = 448;
+  static constexpr int HALF = BM / 2;               // query columns per compute warpgroup
+  static constexpr int NCH = HALF / 32;             // 32-column chunks per compute warpgroup
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;
@@ -82,11 +89,13 @@ struct BwdLayout {
 enum : int {
   SITE_BWD_LOAD_EMPTY = 21, SITE_BWD_LOAD_DRAIN = 22, SITE_BWD_MMA_KV = 23, SITE_BWD_MMA_Q = 24,
   SITE_BWD_MMA_DS = 25, SITE_BWD_MMA_DQE = 26, SITE_BWD_MMA_FIN = 27, SITE_BWD_C_Q = 28,
-  SITE_BWD_C_SDP = 29, SITE_BWD_C_DQ = 30, SITE_BWD_C_DONE = 31, SITE_BWD_DQ = 32
+  SITE_BWD_C_S = 29, SITE_BWD_C_DQ = 30, SITE_BWD_C_DONE = 31, SITE_BWD_DQ = 32,
+  SITE_BWD_MMA_P = 33, SITE_BWD_C_DP = 34
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+// 14 warps: some SM sub-partitions hold four of them, which caps registers at 128 per thread.
+__global__ void __launch_bounds__(448, 1)
 fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
@@ -100,8 +109,10 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint64_t* bar_kv = bars;
   uint64_t* bar_qf = bars + 1;
   uint64_t* bar_qe = bar_qf + L::QST;
-  uint64_t* bar_sdp = bar_qe + L::QST;
-  uint64_t* bar_ds = bar_sdp + 1;
+  uint64_t* bar_s = bar_qe + L::QST;
+  uint64_t* bar_dp = bar_s + 1;
+  uint64_t* bar_p = bar_dp + 1;
+  uint64_t* bar_ds = bar_p + 1;
   uint64_t* bar_dqf = bar_ds + 1;
   uint64_t* bar_dqe = bar_dqf + 2;
   uint64_t* bar_done = bar_dqe + 2;
@@ -143,8 +154,10 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&bar_qf[s], 1);
       mbar_init(&bar_qe[s], 1);
     }
-    mbar_init(bar_sdp, 1);
-    mbar_init(bar_ds, 128);
+    mbar_init(bar_s, 1);
+    mbar_init(bar_dp, 1);
+    mbar_init(bar_p, 256);
+    mbar_init(bar_ds, 256);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_dqf[i], 1);
       mbar_init(&bar_dqe[i], 128);
@@ -154,7 +167,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, L::TMEM_COLS);
     tmem_relinquish();
   }
@@ -163,7 +176,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && n_steps > 0) {
       tma_prefetch_desc(&tm_q);
@@ -199,9 +212,11 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       for (int r = max(0, t - L::QST); r < t; ++r)
         mbar_wait(&bar_qf[r % L::QST], (r / L::QST) & 1, abort_flag, SITE_BWD_LOAD_DRAIN);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_steps > 0) {
+    // The whole warp walks the loop (descriptors stay warp-uniform); one elected lane issues
+    // the MMAs four at a time.
+    if (n_steps > 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, BM, false, false);
       constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, false, true);
       constexpr uint32_t idesc_q = idesc_bf16_f32(128, 64, true, true);
@@ -210,87 +225,125 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint32_t q_addr = smem_u32(smem + L::OFF_Q);
       const uint32_t do_addr = smem_u32(smem + L::OFF_DO);
       const uint32_t ds_addr = smem_u32(smem + L::OFF_DS);
-      // X^T = A B^T over D: A = K or V tile (128 rows), B = Q or dO tile (BM rows), K-major.
-      auto mma_scores = [&](uint32_t a_base, uint32_t b_base, uint32_t d_col) {
+      // K-major views (scores), MN-major views (gradients and dQ).
+      const uint64_t k_kd = sdesc_sw128(k_addr, 16, 1024);
+      const uint64_t v_kd = sdesc_sw128(v_addr, 16, 1024);
+      const uint64_t q_kd = sdesc_sw128(q_addr, 16, 1024);
+      const uint64_t do_kd = sdesc_sw128(do_addr, 16, 1024);
+      const uint64_t q_mn = sdesc_sw128(q_addr, L::Q_SUBTILE, 1024);
+      const uint64_t do_mn = sdesc_sw128(do_addr, L::Q_SUBTILE, 1024);
+      const uint64_t k_mn = sdesc_sw128(k_addr, L::KV_SUBTILE, 1024);
+      const uint64_t ds_mn = sdesc_sw128(ds_addr, L::DS_IBLK, 1024);
+      auto off16 = [](int bytes) -> uint64_t { return static_cast<uint64_t>(bytes >> 4); };
+      // X^T = A B^T over D: A = K or V (128 rows), B = Q or dO of stage st (BM rows), K-major.
+      auto mma_scores = [&](uint64_t a_desc, uint64_t b_desc, int st, uint32_t d_col) {
+        const uint64_t bst = b_desc + off16(st * L::Q_TILE);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const int sub = k >> 2, kk = k & 3;
-          const uint64_t ad = sdesc_sw128(a_base + sub * L::KV_SUBTILE + kk * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(b_base + sub * L::Q_SUBTILE + kk * 32, 16, 1024);
-          mma_ss(tmem + d_col, ad, bd, idesc_s, k > 0 ? 1u : 0u);
+        for (int kb = 0; kb < D / 64; ++kb) {
+          uint64_t a[4], b[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int k = 4 * kb + i;
+            a[i] = a_desc + off16((k >> 2) * L::KV_SUBTILE + (k & 3) * 32);
+            b[i] = bst + off16((k >> 2) * L::Q_SUBTILE + (k & 3) * 32);
+          }
+          mma_ss_x4(tmem + d_col, a, b, idesc_s, kb > 0 ? 1u : 0u);
         }
       };
-      // G += X^T(TMEM, bf16) B over BM rows: B = dO or Q tile, MN-major.
-      auto mma_grad = [&](uint32_t a_col, uint32_t b_base, uint32_t d_col, bool acc) {
+      // G += X^T(TMEM, bf16) B over BM rows: B = dO or Q of stage st, MN-major.  Query columns
+      // [16k, 16k+16) of X^T were written by compute warpgroup h = 16k / HALF into the front
+      // half of its own columns, hence the per-step TMEM column.
+      auto mma_grad = [&](uint32_t a_col, uint64_t b_desc, int st, uint32_t d_col, bool acc) {
+        const uint64_t bst = b_desc + off16(st * L::Q_TILE);
 #pragma unroll
-        for (int k = 0; k < BM / 16; ++k) {
-          const uint64_t bd = sdesc_sw128(b_base + k * 2048, L::Q_SUBTILE, 1024);
-          mma_ts(tmem + d_col, tmem + a_col + k * 8, bd, idesc_g, (acc || k > 0) ? 1u : 0u);
+        for (int kb = 0; kb < BM / 64; ++kb) {
+          uint32_t a[4];
+          uint64_t b[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int k = 4 * kb + i;
+            const uint32_t h = static_cast<uint32_t>((16 * k) / L::HALF);
+            a[i] = tmem + a_col + 8u * k + h * (L::HALF / 2);
+            b[i] = bst + off16(k * 2048);
+          }
+          mma_ts_x4(tmem + d_col, a, b, idesc_g, (acc || kb > 0) ? 1u : 0u);
         }
       };
       auto mma_dq = [&](int buf) {
-        const uint32_t ds = ds_addr + buf * L::DS_TILE;
+        const uint64_t ds = ds_mn + off16(buf * L::DS_TILE);
 #pragma unroll
-        for (int k = 0; k < L::BN / 16; ++k) {
-          uint64_t ad, bd;
-          if constexpr (D == 64) {  // dQ = dS K: A = dS (i contiguous), B = K (d contiguous)
-            ad = sdesc_sw128(ds + k * 2048, L::DS_IBLK, 1024);
-            bd = sdesc_sw128(k_addr + k * 2048, L::KV_SUBTILE, 1024);
-          } else {                  // dQ^T = K^T dS^T: A = K^T (d contiguous), B = dS^T
-            ad = sdesc_sw128(k_addr + k * 2048, L::KV_SUBTILE, 1024);
-            bd = sdesc_sw128(ds + k * 2048, L::DS_IBLK, 1024);
+        for (int kb = 0; kb < L::BN / 64; ++kb) {
+          uint64_t a[4], b[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int k = 4 * kb + i;
+            if constexpr (D == 64) {  // dQ = dS K: A = dS (i contiguous), B = K (d contiguous)
+              a[i] = ds + off16(k * 2048);
+              b[i] = k_mn + off16(k * 2048);
+            } else {                  // dQ^T = K^T dS^T: A = K^T (d contiguous), B = dS^T
+              a[i] = k_mn + off16(k * 2048);
+              b[i] = ds + off16(k * 2048);
+            }
           }
-          mma_ss(tmem + L::DQ_COL + buf * 64, ad, bd, idesc_q, k > 0 ? 1u : 0u);
+          mma_ss_x4(tmem + L::DQ_COL + buf * 64, a, b, idesc_q, kb > 0 ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(bar_kv, 0, abort_flag, SITE_BWD_MMA_KV);
-      ok = ok && mbar_wait(&bar_qf[0], 0, abort_flag, SITE_BWD_MMA_Q);
+      bool ok = mbar_wait_w(bar_kv, 0, abort_flag, SITE_BWD_MMA_KV);
+      ok = ok && mbar_wait_w(&bar_qf[0], 0, abort_flag, SITE_BWD_MMA_Q);
       tc_fence_after();
       if (ok) {
-        mma_scores(k_addr, q_addr, L::S_COL);
-        mma_scores(v_addr, do_addr, L::DP_COL);
-        mma_commit(bar_sdp);
+        mma_scores(k_kd, q_kd, 0, L::S_COL);
+        mma_commit_w(bar_s);
+        mma_scores(v_kd, do_kd, 0, L::DP_COL);
+        mma_commit_w(bar_dp);
       }
       for (int t = 0; ok && t < n_steps; ++t) {
         const int st = t % L::QST;
         const int buf = t & 1;
-        if (!mbar_wait(bar_ds, t & 1, abort_flag, SITE_BWD_MMA_DS)) { ok = false; break; }
-        tc_fence_after();
-        mma_grad(L::S_COL, do_addr + st * L::Q_TILE, L::DV_COL, t > 0);
         const bool next = t + 1 < n_steps;
         const int st1 = (t + 1) % L::QST;
+        if (!mbar_wait_w(bar_p, t & 1, abort_flag, SITE_BWD_MMA_P)) { ok = false; break; }
+        tc_fence_after();
+        mma_grad(L::S_COL, do_mn, st, L::DV_COL, t > 0);
         if (next) {
-          if (!mbar_wait(&bar_qf[st1], ((t + 1) / L::QST) & 1, abort_flag, SITE_BWD_MMA_Q)) {
+          if (!mbar_wait_w(&bar_qf[st1], ((t + 1) / L::QST) & 1, abort_flag, SITE_BWD_MMA_Q)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          mma_scores(k_addr, q_addr + st1 * L::Q_TILE, L::S_COL);
+          mma_scores(k_kd, q_kd, st1, L::S_COL);
+          mma_commit_w(bar_s);
         }
-        mma_grad(L::DP_COL, q_addr + st * L::Q_TILE, L::DK_COL, t > 0);
+        if (!mbar_wait_w(bar_ds, t & 1, abort_flag, SITE_BWD_MMA_DS)) { ok = false; break; }
+        tc_fence_after();
+        mma_grad(L::DP_COL, q_mn, st, L::DK_COL, t > 0);
+        mma_commit_w(&bar_qe[st]);  // Q(t), dO(t), lse(t), Dvec(t) are no longer read after dK(t)
         if (next) {
-          mma_scores(v_addr, do_addr + st1 * L::Q_TILE, L::DP_COL);
-          mma_commit(bar_sdp);
+          mma_scores(v_kd, do_kd, st1, L::DP_COL);
+          mma_commit_w(bar_dp);
         }
-        if (t >= 2 && !mbar_wait(&bar_dqe[buf], ((t - 2) >> 1) & 1, abort_flag, SITE_BWD_MMA_DQE)) {
+        if (t >= 2 &&
+            !mbar_wait_w(&bar_dqe[buf], ((t - 2) >> 1) & 1, abort_flag, SITE_BWD_MMA_DQE)) {
           ok = false;
           break;
         }
         tc_fence_after();
         mma_dq(buf);
-        mma_commit(&bar_dqf[buf]);
-        mma_commit(&bar_qe[st]);
+        mma_commit_w(&bar_dqf[buf]);
       }
-      mma_commit(bar_done);
-      mma_commit(bar_fin);
-      mbar_wait(bar_fin, 0, abort_flag, SITE_BWD_MMA_FIN);
+      mma_commit_w(bar_done);
+      mma_commit_w(bar_fin);
+      mbar_wait_w(bar_fin, 0, abort_flag, SITE_BWD_MMA_FIN);
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------------ compute warpgroup
+  } else if (warp < 8) {
+    // ------------------------------------------------------------------ compute warpgroups
+    const int h = warp >> 2;                  // which half of the query columns
     const int qw = warp & 3;
     const int jl = 32 * qw + lane;            // key row within the tile (= TMEM lane)
     const int kj = k0 + jl;                   // key index
     const uint32_t t_lane = static_cast<uint32_t>(32 * qw) << 16;
+    const uint32_t s_cols = tmem + t_lane + L::S_COL + h * L::HALF;    // my S^T columns
+    const uint32_t dp_cols = tmem + t_lane + L::DP_COL + h * L::HALF;  // my dP^T columns
     const float scale2 = p.scale2;
     bool ok = true;
     int t = 0;
@@ -299,43 +352,91 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int st = t % L::QST;
       const int buf = t & 1;
       const int i0 = it * BM;
+      const int c0 = h * L::HALF;             // first query column of this warpgroup
       bool got = mbar_wait(&bar_qf[st], (t / L::QST) & 1, abort_flag, SITE_BWD_C_Q);
-      got = got && mbar_wait(bar_sdp, t & 1, abort_flag, SITE_BWD_C_SDP);
+      got = got && mbar_wait(bar_s, t & 1, abort_flag, SITE_BWD_C_S);
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      tc_fence_after();
+      const float4* lse4 = reinterpret_cast<const float4*>(s_lse + st * BM + c0);
+      const float4* dv4 = reinterpret_cast<const float4*>(s_dvec + st * BM + c0);
+      const bool edge = (k0 + 128 > kvlen) || (p.causal && k0 + 32 * qw + 31 > i0 + c0);
+      // ---- P = 2^(s*scale2 - lse2), written to TMEM in bf16.  For dS it is kept in fp32 when
+      // one 32-column chunk per thread fits the register budget (d = 128), else as the same
+      // bf16 pairs that feed the dV MMA (d = 64).
+      constexpr bool kP32 = L::NCH == 1;
+      float pf[kP32 ? 32 : 1];
+      uint32_t pk[L::NCH][16];
+#pragma unroll
+      for (int c = 0; c < L::NCH; ++c) {
+        uint32_t sr[32];
+        tmem_ld32(s_cols + 32 * c, sr);
+        tmem_ld_wait();
+        reg_fence(sr);
+        float pv[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 l4 = lse4[8 * c + u];
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 4 * u + e;
+            float pe = ex2_approx(fmaf(__uint_as_float(sr[i]), scale2, -lv[e]));
+            if (edge) {
+              const int qi = i0 + c0 + 32 * c + i;
+              if (kj >= kvlen || (p.causal && kj > qi)) pe = 0.f;
+            }
+            pv[i] = pe;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[c][i] = pack_bf16x2(pv[2 * i], pv[2 * i + 1]);
+        if constexpr (kP32) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pf[i] = pv[i];
+        }
+        tmem_st16(s_cols + 16 * c, pk[c]);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_p);
+      // ---- dS = P (dP - Dvec): bf16 into TMEM (over my dP^T) and into smem for the dQ MMA
+      got = mbar_wait(bar_dp, t & 1, abort_flag, SITE_BWD_C_DP);
       if (t >= 2) got = got && mbar_wait(&bar_dqf[buf], ((t - 2) >> 1) & 1, abort_flag, SITE_BWD_C_DQ);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
-      const float* lse_s = s_lse + st * BM;
-      const float* dv_s = s_dvec + st * BM;
-      const bool edge = (k0 + 128 > kvlen) || (p.causal && k0 + 32 * qw + 31 > i0);
       uint8_t* ds_row = smem + L::OFF_DS + buf * L::DS_TILE + jl * 128;
-#pragma unroll 1
-      for (int cc = 0; cc < BM / 32; ++cc) {
-        uint32_t s[32], dp[32];
-        tmem_ld32(tmem + t_lane + L::S_COL + 32 * cc, s);
-        tmem_ld32(tmem + t_lane + L::DP_COL + 32 * cc, dp);
+#pragma unroll
+      for (int c = 0; c < L::NCH; ++c) {
+        uint32_t dr[32];
+        tmem_ld32(dp_cols + 32 * c, dr);
         tmem_ld_wait();
-        reg_fence(s);
-        reg_fence(dp);
-        uint32_t pp[16], dd[16];
+        reg_fence(dr);
+        float dsv[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float pv[2], dsv[2];
+        for (int u = 0; u < 8; ++u) {
+          const float4 d4 = dv4[8 * c + u];
+          const float dvv[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int col = 32 * cc + 2 * i + h;
-            float pe = ex2_approx(fmaf(__uint_as_float(s[2 * i + h]), scale2, -lse_s[col]));
-            if (edge && (kj >= kvlen || (p.causal && kj > i0 + col))) pe = 0.f;
-            pv[h] = pe;
-            dsv[h] = pe * (__uint_as_float(dp[2 * i + h]) - dv_s[col]);
+          for (int e = 0; e < 4; ++e) {
+            const int i = 4 * u + e;
+            float pe;
+            if constexpr (kP32) {
+              pe = pf[i];
+            } else {
+              const uint32_t w = pk[c][i >> 1];
+              pe = __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
+            }
+            dsv[i] = pe * (__uint_as_float(dr[i]) - dvv[e]);
           }
-          pp[i] = pack_bf16x2(pv[0], pv[1]);
-          dd[i] = pack_bf16x2(dsv[0], dsv[1]);
         }
-        tmem_st16(tmem + t_lane + L::S_COL + 16 * cc, pp);
-        tmem_st16(tmem + t_lane + L::DP_COL + 16 * cc, dd);
-        // dS^T row jl, columns 32cc..32cc+31 -> 4 swizzled 16-byte chunks
-        const int iblk = (32 * cc) >> 6;
-        const int chunk0 = ((32 * cc) & 63) >> 3;
+        uint32_t dd[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) dd[i] = pack_bf16x2(dsv[2 * i], dsv[2 * i + 1]);
+        tmem_st16(dp_cols + 16 * c, dd);
+        // dS^T row jl, query columns c0+32c .. +31 -> 4 swizzled 16-byte chunks
+        const int col = c0 + 32 * c;
+        const int iblk = col >> 6;
+        const int chunk0 = (col & 63) >> 3;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int pos = (chunk0 + u) ^ (jl & 7);
@@ -350,39 +451,36 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       ++t;
     }
     // ---------------------------------------------------------------- epilogue: dK, dV
+    // warpgroup 0 writes dV, warpgroup 1 writes dK (x scale)
     if (ok && n_steps > 0) {
       const bool got = mbar_wait(bar_done, 0, abort_flag, SITE_BWD_C_DONE);
       ok = __all_sync(0xffffffffu, got);
       tc_fence_after();
     }
-    if (ok && k0 < N) {
-#pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t col0 = which == 0 ? L::DV_COL : L::DK_COL;
-        const float mul = which == 0 ? 1.0f : p.scale;
-        __nv_bfloat16* dst_row =
-            (which == 0 ? p.dv : p.dk) + (static_cast<size_t>(bh) * N + kj) * D;
+    if (ok) {
+      const uint32_t col0 = h == 0 ? L::DV_COL : L::DK_COL;
+      const float mul = h == 0 ? 1.0f : p.scale;
+      __nv_bfloat16* dst_row = (h == 0 ? p.dv : p.dk) + (static_cast<size_t>(bh) * N + kj) * D;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t g[32];
-          if (n_steps > 0) {
-            tmem_ld32(tmem + t_lane + col0 + 32 * c, g);
-            tmem_ld_wait();
-            reg_fence(g);
-          } else {
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t g[32];
+        if (n_steps > 0) {
+          tmem_ld32(tmem + t_lane + col0 + 32 * c, g);
+          tmem_ld_wait();
+          reg_fence(g);
+        } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) g[i] = 0u;
-          }
-          uint32_t h[16];
+          for (int i = 0; i < 32; ++i) g[i] = 0u;
+        }
+        uint32_t hv[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            h[i] = pack_bf16x2(__uint_as_float(g[2 * i]) * mul, __uint_as_float(g[2 * i + 1]) * mul);
-          if (kj < N) {
-            uint4* dst = reinterpret_cast<uint4*>(dst_row + 32 * c);
+        for (int i = 0; i < 16; ++i)
+          hv[i] = pack_bf16x2(__uint_as_float(g[2 * i]) * mul, __uint_as_float(g[2 * i + 1]) * mul);
+        if (kj < N) {
+          uint4* dst = reinterpret_cast<uint4*>(dst_row + 32 * c);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
-          }
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
         }
       }
     }
@@ -433,7 +531,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);
   }

@@ -12,8 +12,11 @@
 // CTA layout (320 threads, one CTA per SM):
 //   warps 0-3  softmax warpgroup for Q tile 0 (rows m0 .. m0+127), one thread per row
 //   warps 4-7  softmax warpgroup for Q tile 1 (rows m0+128 .. m0+255)
-//   warp  8    TMA producer: Q once, then K/V tiles of 128 keys through a STAGES-deep ring
-//   warp  9    MMA issuer (one thread): S_w = Q_w K^T into TMEM, O_w += P_w V from TMEM P
+//   warp  8    TMA producer: Q once, then K and V tiles of 128 keys through separate rings
+//              (a K stage frees as soon as both S MMAs of its tile finish, a V stage after
+//              both PV MMAs, so K runs further ahead than a shared ring would allow)
+//   warp  9    MMA issuer (whole warp, one elected lane issues): S_w = Q_w K^T into TMEM,
+//              O_w += P_w V with P taken from TMEM
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [256+D,256+2D).
 // P_w (bf16, two per 32-bit column) overwrites columns [0,64) of S_w after the softmax
 // warpgroup has read S_w into registers.
@@ -49,15 +52,17 @@ template <int D>
 struct FwdLayout {
   static constexpr int BM = 128;                    // query rows per Q tile
   static constexpr int BN = 128;                    // keys per KV tile
-  static constexpr int STAGES = D == 64 ? 4 : 2;
+  static constexpr int KST = D == 64 ? 5 : 3;       // K ring depth
+  static constexpr int VST = D == 64 ? 4 : 2;       // V ring depth
   static constexpr int SUB = D / 64;                // 64-column (128-byte) sub-tiles
   static constexpr int SUBTILE = 128 * 128;         // bytes of one 128-row x 64-col sub-tile
   static constexpr int TILE = 128 * D * 2;          // bytes of one 128-row tile
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * TILE;
-  static constexpr int OFF_V = OFF_K + STAGES * TILE;
-  static constexpr int OFF_BAR = OFF_V + STAGES * TILE;
-  static constexpr int NBAR = 1 + 3 * STAGES + 6 + 1;
+  static constexpr int OFF_V = OFF_K + KST * TILE;
+  static constexpr int OFF_BAR = OFF_V + VST * TILE;
+  // q, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], p_full[2], o_done[2], fin
+  static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 6 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;   // slack for 1024-byte alignment
@@ -85,9 +90,10 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* bar_q = bars;
   uint64_t* bar_kf = bars + 1;
-  uint64_t* bar_vf = bar_kf + L::STAGES;
-  uint64_t* bar_ke = bar_vf + L::STAGES;
-  uint64_t* bar_sf = bar_ke + L::STAGES;
+  uint64_t* bar_ke = bar_kf + L::KST;
+  uint64_t* bar_vf = bar_ke + L::KST;
+  uint64_t* bar_ve = bar_vf + L::VST;
+  uint64_t* bar_sf = bar_ve + L::VST;
   uint64_t* bar_pf = bar_sf + 2;
   uint64_t* bar_od = bar_pf + 2;
   uint64_t* bar_fin = bar_od + 2;
@@ -127,10 +133,13 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
-    for (int s = 0; s < L::STAGES; ++s) {
+    for (int s = 0; s < L::KST; ++s) {
       mbar_init(&bar_kf[s], 1);
-      mbar_init(&bar_vf[s], 1);
       mbar_init(&bar_ke[s], 1);
+    }
+    for (int s = 0; s < L::VST; ++s) {
+      mbar_init(&bar_vf[s], 1);
+      mbar_init(&bar_ve[s], 1);
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&bar_sf[w], 1);
@@ -162,109 +171,127 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int s = 0; s < L::SUB; ++s)
           tma_load_3d(smem + L::OFF_Q + w * L::TILE + s * L::SUBTILE, &tm_q, bar_q, s * 64,
                       m0 + 128 * w, bh);
-      int it = 0;
+      int kn = 0, vn = 0;  // K and V tiles issued so far
       for (int j = 0; j < j_end; ++j) {
         if (flags_of(j) == 0) continue;
-        const int st = it % L::STAGES;
-        if (it >= L::STAGES &&
-            !mbar_wait(&bar_ke[st], ((it / L::STAGES) - 1) & 1, abort_flag, SITE_FWD_LOAD_EMPTY))
+        const int ks = kn % L::KST, vs = vn % L::VST;
+        if (kn >= L::KST &&
+            !mbar_wait(&bar_ke[ks], ((kn / L::KST) - 1) & 1, abort_flag, SITE_FWD_LOAD_EMPTY))
           break;
-        mbar_arrive_expect_tx(&bar_kf[st], L::TILE);
+        mbar_arrive_expect_tx(&bar_kf[ks], L::TILE);
         for (int s = 0; s < L::SUB; ++s)
-          tma_load_3d(smem + L::OFF_K + st * L::TILE + s * L::SUBTILE, &tm_k, &bar_kf[st], s * 64,
+          tma_load_3d(smem + L::OFF_K + ks * L::TILE + s * L::SUBTILE, &tm_k, &bar_kf[ks], s * 64,
                       j * 128, bh);
-        mbar_arrive_expect_tx(&bar_vf[st], L::TILE);
+        ++kn;
+        if (vn >= L::VST &&
+            !mbar_wait(&bar_ve[vs], ((vn / L::VST) - 1) & 1, abort_flag, SITE_FWD_LOAD_EMPTY))
+          break;
+        mbar_arrive_expect_tx(&bar_vf[vs], L::TILE);
         for (int s = 0; s < L::SUB; ++s)
-          tma_load_3d(smem + L::OFF_V + st * L::TILE + s * L::SUBTILE, &tm_v, &bar_vf[st], s * 64,
+          tma_load_3d(smem + L::OFF_V + vs * L::TILE + s * L::SUBTILE, &tm_v, &bar_vf[vs], s * 64,
                       j * 128, bh);
-        ++it;
+        ++vn;
       }
       // Never leave the CTA with a copy in flight: wait for the last loads of every stage
       // (immediate in the normal path, where the MMA thread consumed them).
       mbar_wait(bar_q, 0, abort_flag, SITE_FWD_LOAD_DRAIN);
-      for (int r = max(0, it - L::STAGES); r < it; ++r) {
-        mbar_wait(&bar_kf[r % L::STAGES], (r / L::STAGES) & 1, abort_flag, SITE_FWD_LOAD_DRAIN);
-        mbar_wait(&bar_vf[r % L::STAGES], (r / L::STAGES) & 1, abort_flag, SITE_FWD_LOAD_DRAIN);
-      }
+      for (int r = max(0, kn - L::KST); r < kn; ++r)
+        mbar_wait(&bar_kf[r % L::KST], (r / L::KST) & 1, abort_flag, SITE_FWD_LOAD_DRAIN);
+      for (int r = max(0, vn - L::VST); r < vn; ++r)
+        mbar_wait(&bar_vf[r % L::VST], (r / L::VST) & 1, abort_flag, SITE_FWD_LOAD_DRAIN);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
-      const uint32_t q_addr = smem_u32(smem + L::OFF_Q);
-      const uint32_t k_addr = smem_u32(smem + L::OFF_K);
-      const uint32_t v_addr = smem_u32(smem + L::OFF_V);
-      bool ok = mbar_wait(bar_q, 0, abort_flag, SITE_FWD_MMA_Q);
+    // The whole warp walks the loop (descriptors stay warp-uniform); one elected lane issues.
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+    // Base descriptors; stage, sub-tile and K-step offsets are added to the start-address
+    // field (16-byte units).  Q/K: K-major, 128-byte rows, 8-row groups 1 KB apart.
+    // V: MN-major, 64-column blocks one sub-tile apart.
+    const uint64_t q_desc = sdesc_sw128(smem_u32(smem + L::OFF_Q), 16, 1024);
+    const uint64_t k_desc = sdesc_sw128(smem_u32(smem + L::OFF_K), 16, 1024);
+    const uint64_t v_desc = sdesc_sw128(smem_u32(smem + L::OFF_V), L::SUBTILE, 1024);
+    auto koff = [](int k) -> uint64_t {  // K-step k of a K-major operand, in 16-byte units
+      return static_cast<uint64_t>(((k >> 2) * L::SUBTILE + (k & 3) * 32) >> 4);
+    };
+    bool ok = mbar_wait_w(bar_q, 0, abort_flag, SITE_FWD_MMA_Q);
+    tc_fence_after();
+    int it = 0;
+    int cnt0 = 0, cnt1 = 0;
+    int prev_flags = 0, prev_vs = 0;
+    // O_w += P_w V(vs): P_w from TMEM (bf16 pairs over S_w), V MN-major.
+    auto issue_pv = [&](int w, int vs, int& cnt) -> bool {
+      if (!mbar_wait_w(&bar_pf[w], cnt & 1, abort_flag, SITE_FWD_MMA_P)) return false;
       tc_fence_after();
-      int it = 0;
-      int cnt[2] = {0, 0};
-      int prev_flags = 0, prev_st = 0;
-      auto issue_pv = [&](int w, int st) -> bool {
-        if (!mbar_wait(&bar_pf[w], cnt[w] & 1, abort_flag, SITE_FWD_MMA_P)) return false;
-        tc_fence_after();
-        const uint32_t a_tmem = tmem + L::s_col(w);
-        const uint32_t d_tmem = tmem + L::O_COL0 + w * D;
+      const uint32_t a_tmem = tmem + L::s_col(w);
+      const uint32_t d_tmem = tmem + L::O_COL0 + w * D;
+      const uint64_t vb = v_desc + static_cast<uint64_t>((vs * L::TILE) >> 4);
 #pragma unroll
-        for (int k = 0; k < L::BN / 16; ++k) {
-          const uint64_t bdesc =
-              sdesc_sw128(v_addr + st * L::TILE + k * 2048, L::SUBTILE, 1024);
-          mma_ts(d_tmem, a_tmem + k * 8, bdesc, idesc_o, (cnt[w] > 0 || k > 0) ? 1u : 0u);
-        }
-        mma_commit(&bar_od[w]);
-        ++cnt[w];
-        return true;
-      };
-      for (int j = 0; ok && j < j_end; ++j) {
-        const int f = flags_of(j);
-        if (f == 0) continue;
-        const int st = it % L::STAGES;
-        if (!mbar_wait(&bar_kf[st], (it / L::STAGES) & 1, abort_flag, SITE_FWD_MMA_K)) { ok = false; break; }
-        if (prev_flags != 0 &&
-            !mbar_wait(&bar_vf[prev_st], ((it - 1) / L::STAGES) & 1, abort_flag, SITE_FWD_MMA_V)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+      for (int kb = 0; kb < L::BN / 64; ++kb) {
+        uint32_t a[4];
+        uint64_t b[4];
 #pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          if (prev_flags & (1 << w)) {
-            if (!issue_pv(w, prev_st)) { ok = false; break; }
-          }
-          if (f & (1 << w)) {
-            const uint32_t d_tmem = tmem + L::s_col(w);
-#pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const int sub = k >> 2, kk = k & 3;
-              const uint64_t adesc =
-                  sdesc_sw128(q_addr + w * L::TILE + sub * L::SUBTILE + kk * 32, 16, 1024);
-              const uint64_t bdesc =
-                  sdesc_sw128(k_addr + st * L::TILE + sub * L::SUBTILE + kk * 32, 16, 1024);
-              mma_ss(d_tmem, adesc, bdesc, idesc_s, k > 0 ? 1u : 0u);
-            }
-            mma_commit(&bar_sf[w]);
-          }
+        for (int i = 0; i < 4; ++i) {
+          const int k = 4 * kb + i;
+          a[i] = a_tmem + 8 * k;
+          b[i] = vb + static_cast<uint64_t>((k * 2048) >> 4);
         }
-        if (!ok) break;
-        if (prev_flags != 0) mma_commit(&bar_ke[prev_st]);
-        prev_flags = f;
-        prev_st = st;
-        ++it;
+        mma_ts_x4(d_tmem, a, b, idesc_o, (cnt > 0 || kb > 0) ? 1u : 0u);
       }
-      if (ok && prev_flags != 0) {
-        if (mbar_wait(&bar_vf[prev_st], ((it - 1) / L::STAGES) & 1, abort_flag, SITE_FWD_MMA_V)) {
-          tc_fence_after();
-          for (int w = 0; w < 2; ++w)
-            if (prev_flags & (1 << w)) {
-              if (!issue_pv(w, prev_st)) break;
-            }
-          mma_commit(&bar_ke[prev_st]);
+      mma_commit_w(&bar_od[w]);
+      ++cnt;
+      return true;
+    };
+    // S_w = Q_w K(ks)^T
+    auto issue_s = [&](int w, int ks) {
+      const uint64_t qa = q_desc + static_cast<uint64_t>((w * L::TILE) >> 4);
+      const uint64_t kb0 = k_desc + static_cast<uint64_t>((ks * L::TILE) >> 4);
+#pragma unroll
+      for (int kb = 0; kb < D / 64; ++kb) {
+        uint64_t a[4], b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          a[i] = qa + koff(4 * kb + i);
+          b[i] = kb0 + koff(4 * kb + i);
         }
+        mma_ss_x4(tmem + L::s_col(w), a, b, idesc_s, kb > 0 ? 1u : 0u);
       }
-      // all MMAs issued by this thread have completed before TMEM is released
-      mma_commit(bar_fin);
-      mbar_wait(bar_fin, 0, abort_flag, SITE_FWD_MMA_FIN);
+      mma_commit_w(&bar_sf[w]);
+    };
+    for (int j = 0; ok && j < j_end; ++j) {
+      const int f = flags_of(j);
+      if (f == 0) continue;
+      const int ks = it % L::KST, vs = it % L::VST;
+      if (!mbar_wait_w(&bar_kf[ks], (it / L::KST) & 1, abort_flag, SITE_FWD_MMA_K)) { ok = false; break; }
+      if (prev_flags != 0 &&
+          !mbar_wait_w(&bar_vf[prev_vs], ((it - 1) / L::VST) & 1, abort_flag, SITE_FWD_MMA_V)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // for w = 0 then 1: PV_w of the previous tile, then S_w of this tile
+      if (prev_flags & 1) ok = ok && issue_pv(0, prev_vs, cnt0);
+      if (ok && (f & 1)) issue_s(0, ks);
+      if (ok && (prev_flags & 2)) ok = issue_pv(1, prev_vs, cnt1);
+      if (ok && (f & 2)) issue_s(1, ks);
+      if (!ok) break;
+      mma_commit_w(&bar_ke[ks]);                          // K(j) read by both S MMAs
+      if (prev_flags != 0) mma_commit_w(&bar_ve[prev_vs]);  // V(prev) read by both PV MMAs
+      prev_flags = f;
+      prev_vs = vs;
+      ++it;
     }
+    if (ok && prev_flags != 0) {
+      if (mbar_wait_w(&bar_vf[prev_vs], ((it - 1) / L::VST) & 1, abort_flag, SITE_FWD_MMA_V)) {
+        tc_fence_after();
+        if (prev_flags & 1) ok = issue_pv(0, prev_vs, cnt0);
+        if (ok && (prev_flags & 2)) ok = issue_pv(1, prev_vs, cnt1);
+        mma_commit_w(&bar_ve[prev_vs]);
+      }
+    }
+    // all MMAs issued by this warp have completed before TMEM is released
+    mma_commit_w(bar_fin);
+    mbar_wait_w(bar_fin, 0, abort_flag, SITE_FWD_MMA_FIN);
   } else {
     // ------------------------------------------------------------------ softmax warpgroups
     const int w = warp >> 2;

@@ -154,6 +154,58 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
       : "memory");
 }
 
+// Warp-collective issue: every lane of the (converged) warp passes identical operands and one
+// lane chosen by elect.sync issues.  Keeping the whole warp on the MMA path lets the compiler
+// hold descriptors in uniform registers; batching four MMAs under one election keeps the
+// single issuing thread ahead of the tensor pipe even for N = 128 tiles.
+// Four MMAs D (+)= A_i * B_i: the first accumulates when acc != 0, the next three always do.
+__device__ __forceinline__ void mma_ss_x4(uint32_t d_tmem, const uint64_t (&a)[4],
+                                          const uint64_t (&b)[4], uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "elect.sync _|q, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %10, 0;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %9, p;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %4, %9, 1;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %6, %9, 1;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %8, %9, 1;\n\t}\n" ::"r"(d_tmem),
+      "l"(a[0]), "l"(b[0]), "l"(a[1]), "l"(b[1]), "l"(a[2]), "l"(b[2]), "l"(a[3]), "l"(b[3]),
+      "r"(idesc), "r"(acc)
+      : "memory");
+}
+// Same with the A operands in TMEM.
+__device__ __forceinline__ void mma_ts_x4(uint32_t d_tmem, const uint32_t (&a)[4],
+                                          const uint64_t (&b)[4], uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "elect.sync _|q, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %10, 0;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %9, p;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %4, %9, 1;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %6, %9, 1;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %8, %9, 1;\n\t}\n" ::"r"(d_tmem),
+      "r"(a[0]), "l"(b[0]), "r"(a[1]), "l"(b[1]), "r"(a[2]), "l"(b[2]), "r"(a[3]), "l"(b[3]),
+      "r"(idesc), "r"(acc)
+      : "memory");
+}
+// Warp-collective commit: one elected lane arrives on `bar` once all MMAs it issued are done.
+// (The elected lane is the same for every election of a converged warp, so it is the lane
+// that issued the MMAs.)
+__device__ __forceinline__ void mma_commit_w(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "elect.sync _|q, 0xffffffff;\n\t"
+      "@q tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+// Warp-uniform bounded wait: true only if every lane saw the phase complete.
+__device__ __forceinline__ bool mbar_wait_w(uint64_t* bar, uint32_t parity,
+                                            volatile int* abort_flag, int site) {
+  const bool got = mbar_wait(bar, parity, abort_flag, site);
+  return __all_sync(0xffffffffu, got);
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
 //   [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format (1 = bf16),
 //   bit 15 / 16: A / B major (0 = K-major, 1 = MN-major), [17,23) N >> 3, [24,29) M >> 4.
