@@ -35,6 +35,7 @@ SIGNATURES = {
     "fa_naive_workspace_size": (_sz, [_i, _i, _i]),
     "fa_naive_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz,
                           _vp]),
+    "fa_diag_exp2": (_i, [_vp, _vp, _vp, _vp, _i, _vp]),
     "fa_get_last_error": (ctypes.c_char_p, []),
     "fa_device_status": (_i, [ctypes.POINTER(ctypes.c_uint)]),
 }
@@ -208,6 +209,16 @@ def naive_fwd(q, k, v, scale: Optional[float] = None, causal: bool = False, bloc
                           int(causal), bm, kl, _ptr(ws), ws.numel(), _stream())
     _check(rc, "fa_naive_fwd")
     return o, l
+
+
+def diag_exp2(x):
+    """(FMA-pipe 2^x, ex2.approx, exp2f) of a float32 CUDA tensor; diagnostic only."""
+    lib = load()
+    _require(x, "x", torch.float32)
+    y = [torch.empty_like(x) for _ in range(3)]
+    rc = lib.fa_diag_exp2(_ptr(x), _ptr(y[0]), _ptr(y[1]), _ptr(y[2]), x.numel(), _stream())
+    _check(rc, "fa_diag_exp2")
+    return tuple(y)
 
 
 def device_status() -> int:

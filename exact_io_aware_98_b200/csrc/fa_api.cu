@@ -276,6 +276,14 @@ int fa_fwd_tile_reference(const void* q, const void* k, const void* v, void* o, 
   return check_launch("fa_fwd_rowwarp_kernel<bf16>");
 }
 
+int fa_diag_exp2(const float* x, float* y_fma, float* y_mufu, float* y_ref, int n, void* stream) {
+  if (!x || !y_fma || !y_mufu || !y_ref) return fail(FA_ERR_INVALID, "null pointer");
+  if (n < 1) return fail(FA_ERR_INVALID, "n must be >= 1");
+  const int blocks = (n + 511) / 512;
+  fa::diag_exp2_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_fma, y_mufu, y_ref, n);
+  return check_launch("diag_exp2_kernel");
+}
+
 size_t fa_naive_workspace_size(int B, int H, int N) {
   if (B < 1 || H < 1 || N < 1) return 0;
   return static_cast<size_t>(B) * H * N * N * 2;

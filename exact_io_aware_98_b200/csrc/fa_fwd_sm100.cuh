@@ -68,6 +68,8 @@ struct FwdLayout {
   static constexpr int SMEM_ALLOC = BYTES + 1024;   // slack for 1024-byte alignment
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t O_COL0 = 256;
+  // one P pair in EMU_EVERY is exponentiated on the FMA pipe (0 = all on MUFU)
+  static constexpr int EMU_EVERY = 4;
   __device__ static constexpr uint32_t s_col(int w) { return static_cast<uint32_t>(w) * 128u; }
 };
 
@@ -329,29 +331,46 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (col >= kvlen || (p.causal && col > row)) r[c][i] = __float_as_uint(-INFINITY);
           }
       }
-      float mx = -INFINITY;
+      // row maximum: eight independent chains of 3-input max
+      float mc[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int u = 0; u < 8; ++u) mc[u] = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(r[c][i]));
+      for (int k = 0; k < 128; k += 2)
+        mc[(k >> 1) & 7] = fmax3(mc[(k >> 1) & 7], __uint_as_float(r[k >> 5][k & 31]),
+                                 __uint_as_float(r[k >> 5][(k & 31) + 1]));
+      const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]),
+                             fmaxf(mc[6], mc[7]));
       const float tmax = mx * scale2;
       float m_new = m_ref;
       if (tmax > m_ref + 8.0f) m_new = tmax;  // also taken when m_ref is still -inf
       const float alpha = (m_new == m_ref) ? 1.0f : ex2_approx(m_ref - m_new);
       const float neg_base = (m_new == -INFINITY) ? 0.0f : -m_new;
-      float rs0 = 0.f, rs1 = 0.f;
+      // P = 2^(s*scale2 - m) in pairs: packed fp32x2 scale-and-shift and row sums (four
+      // independent accumulator pairs).  On tiles without masked elements, one pair in
+      // L::EMU_EVERY takes 2^x on the FMA pipe instead of MUFU, which the other pairs keep busy.
+      float ra[4] = {0.f, 0.f, 0.f, 0.f}, rb[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[4][16];
+      auto exp_pairs = [&](bool use_fma) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(r[c][2 * i]), scale2, neg_base));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(r[c][2 * i + 1]), scale2, neg_base));
-          rs0 += p0;
-          rs1 += p1;
+        for (int q = 0; q < 64; ++q) {
+          const int c = q >> 4, i = q & 15;
+          float x0, x1, p0, p1;
+          ffma2(x0, x1, __uint_as_float(r[c][2 * i]), __uint_as_float(r[c][2 * i + 1]), scale2,
+                scale2, neg_base, neg_base);
+          if (use_fma && L::EMU_EVERY > 0 && (q % L::EMU_EVERY) == L::EMU_EVERY - 1) {
+            exp2_fma2(p0, p1, x0, x1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          fadd2(ra[q & 3], rb[q & 3], ra[q & 3], rb[q & 3], p0, p1);
           pk[c][i] = pack_bf16x2(p0, p1);
         }
-      l = alpha * l + (rs0 + rs1);
+      };
+      if (edge) exp_pairs(false);  // masked elements are -inf: MUFU gives exact zeros
+      else exp_pairs(true);
+      l = alpha * l + ((ra[0] + ra[1]) + (ra[2] + ra[3]) + ((rb[0] + rb[1]) + (rb[2] + rb[3])));
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_st16(t_s + 16 * c, pk[c]);
       const bool rescale = (cnt > 0) && (m_new != m_ref);

@@ -15,6 +15,8 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace fa {
 
 template <typename T> __device__ __forceinline__ float to_f(T x);
@@ -261,6 +263,27 @@ dq_convert_kernel(const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ 
     *reinterpret_cast<uint4*>(dq + e) = u;
   } else {
     for (long long x = e; x < n; ++x) dq[x] = __float2bfloat16_rn(dq_acc[x] * scale);
+  }
+}
+
+// Diagnostic: the two exp2 paths of the forward softmax side by side, for their tests.
+__global__ void __launch_bounds__(256)
+diag_exp2_kernel(const float* __restrict__ x, float* __restrict__ y_fma, float* __restrict__ y_mufu,
+                 float* __restrict__ y_ref, int n) {
+  const int i = (blockIdx.x * 256 + threadIdx.x) * 2;
+  if (i + 1 < n) {
+    float a, b;
+    exp2_fma2(a, b, x[i], x[i + 1]);
+    y_fma[i] = a;
+    y_fma[i + 1] = b;
+  } else if (i < n) {
+    float a, b;
+    exp2_fma2(a, b, x[i], 0.0f);
+    y_fma[i] = a;
+  }
+  for (int k = i; k < min(i + 2, n); ++k) {
+    y_mufu[k] = ex2_approx(x[k]);
+    y_ref[k] = exp2f(x[k]);
   }
 }
 

@@ -303,4 +303,52 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// ----------------------------------------------------------------------------- packed fp32 math
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// (d0, d1) = (a0 * b0 + c0, a1 * b1 + c1), one packed fp32x2 instruction
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                      float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+// (d0, d1) = (a0 + b0, a1 + b1)
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// 2^x on the FMA pipe, for a pair, x <= 126 (x below -126 returns a value below 2^-125).
+// Cody-Waite style reduction x = n + f, n = round(x), |f| <= 1/2, via the 1.5*2^23 rounding
+// constant; 2^f by a cubic with constant term 1 whose other coefficients were fitted here
+// (Lawson-weighted least squares for minimal relative error on [-1/2, 1/2]: max relative
+// error 1.0e-4, below the 2^-9 rounding of the bf16 P it feeds); 2^n is added to the exponent
+// field with an integer add (the low 23 bits of the rounding constant's exponent part vanish
+// under the shift, so bits(x + 1.5*2^23) << 23 == n << 23).
+__device__ __forceinline__ void exp2_fma2(float& y0, float& y1, float x0, float x1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float kC1 = 0.6932829f, kC2 = 0.24221037f, kC3 = 0.05500858f;
+  x0 = fmaxf(x0, -126.0f);
+  x1 = fmaxf(x1, -126.0f);
+  float j0, j1, n0, n1, f0, f1, p0, p1;
+  fadd2(j0, j1, x0, x1, kRound, kRound);
+  fadd2(n0, n1, j0, j1, -kRound, -kRound);
+  ffma2(f0, f1, n0, n1, -1.0f, -1.0f, x0, x1);
+  ffma2(p0, p1, kC3, kC3, f0, f1, kC2, kC2);
+  ffma2(p0, p1, p0, p1, f0, f1, kC1, kC1);
+  ffma2(p0, p1, p0, p1, f0, f1, 1.0f, 1.0f);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(j0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(j1) << 23));
+}
+
 }  // namespace fa

@@ -133,6 +133,15 @@ int fa_naive_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  int N, int d, float scale, int causal, const uint8_t* block_mask,
                  const int32_t* kv_len, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * fa_diag_exp2 -- diagnostic for the two ways the forward softmax evaluates 2^x: y_fma gets the
+ * FMA-pipe evaluation (rounding reduction x = n + f, |f| <= 1/2, a cubic for 2^f with constant
+ * term 1 fitted for minimal relative error, and 2^n added to the exponent bits; relative error
+ * below 1.1e-4 for -125 <= x <= 126), y_mufu the hardware ex2.approx, y_ref CUDA's exp2f.
+ * x, y_fma, y_mufu, y_ref: device float arrays of n elements.  Asynchronous on `stream`.
+ */
+int fa_diag_exp2(const float* x, float* y_fma, float* y_mufu, float* y_ref, int n, void* stream);
+
 /* Message for the most recent non-OK status returned on this host thread. */
 const char* fa_get_last_error(void);
 
