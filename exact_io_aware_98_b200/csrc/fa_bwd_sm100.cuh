@@ -74,6 +74,7 @@ struct BwdLayout {
   static constexpr int THREADS = 448;
   static constexpr int HALF = BM / 2;               // query columns per compute warpgroup
   static constexpr int NCH = HALF / 32;             // 32-column chunks per compute warpgroup
+  static constexpr int EMU_EVERY = 0;               // one P pair in EMU_EVERY exponentiated on FMA (0: none)
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;
@@ -373,21 +374,39 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         tmem_ld_wait();
         reg_fence(sr);
         float pv[32];
+        // x = s*scale2 - lse2 in packed pairs; on tiles without masked keys one pair in
+        // L::EMU_EVERY takes 2^x on the FMA pipe, the rest on MUFU
+        auto p_chunk = [&](bool masked) {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float4 l4 = lse4[8 * c + u];
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+          for (int u = 0; u < 8; ++u) {
+            const float4 l4 = lse4[8 * c + u];
+            float x[4];
+            ffma2(x[0], x[1], __uint_as_float(sr[4 * u]), __uint_as_float(sr[4 * u + 1]), scale2,
+                  scale2, -l4.x, -l4.y);
+            ffma2(x[2], x[3], __uint_as_float(sr[4 * u + 2]), __uint_as_float(sr[4 * u + 3]), scale2,
+                  scale2, -l4.z, -l4.w);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = 4 * u + e;
-            float pe = ex2_approx(fmaf(__uint_as_float(sr[i]), scale2, -lv[e]));
-            if (edge) {
-              const int qi = i0 + c0 + 32 * c + i;
-              if (kj >= kvlen || (p.causal && kj > qi)) pe = 0.f;
+            for (int hp = 0; hp < 2; ++hp) {
+              const int i = 4 * u + 2 * hp;
+              float p0, p1;
+              if (!masked && L::EMU_EVERY > 0 && ((i >> 1) % L::EMU_EVERY) == L::EMU_EVERY - 1) {
+                exp2_fma2(p0, p1, x[2 * hp], x[2 * hp + 1]);
+              } else {
+                p0 = ex2_approx(x[2 * hp]);
+                p1 = ex2_approx(x[2 * hp + 1]);
+              }
+              if (masked) {
+                const int qi = i0 + c0 + 32 * c + i;
+                if (kj >= kvlen || (p.causal && kj > qi)) p0 = 0.f;
+                if (kj >= kvlen || (p.causal && kj > qi + 1)) p1 = 0.f;
+              }
+              pv[i] = p0;
+              pv[i + 1] = p1;
             }
-            pv[i] = pe;
           }
-        }
+        };
+        if (edge) p_chunk(true);
+        else p_chunk(false);
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[c][i] = pack_bf16x2(pv[2 * i], pv[2 * i + 1]);
         if constexpr (kP32) {
