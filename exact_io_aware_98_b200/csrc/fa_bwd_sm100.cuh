@@ -389,7 +389,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             for (int hp = 0; hp < 2; ++hp) {
               const int i = 4 * u + 2 * hp;
               float p0, p1;
-              if (!masked && L::EMU_EVERY > 0 && ((i >> 1) % L::EMU_EVERY) == L::EMU_EVERY - 1) {
+              if (!masked && L::EMU_EVERY > 0 && ((i >> 1) % (L::EMU_EVERY > 0 ? L::EMU_EVERY : 1)) == L::EMU_EVERY - 1) {
                 exp2_fma2(p0, p1, x[2 * hp], x[2 * hp + 1]);
               } else {
                 p0 = ex2_approx(x[2 * hp]);

@@ -358,7 +358,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           float x0, x1, p0, p1;
           ffma2(x0, x1, __uint_as_float(r[c][2 * i]), __uint_as_float(r[c][2 * i + 1]), scale2,
                 scale2, neg_base, neg_base);
-          if (use_fma && L::EMU_EVERY > 0 && (q % L::EMU_EVERY) == L::EMU_EVERY - 1) {
+          if (use_fma && L::EMU_EVERY > 0 && (q % (L::EMU_EVERY > 0 ? L::EMU_EVERY : 1)) == L::EMU_EVERY - 1) {
             exp2_fma2(p0, p1, x0, x1);
           } else {
             p0 = ex2_approx(x0);
