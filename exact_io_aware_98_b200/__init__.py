@@ -36,6 +36,7 @@ SIGNATURES = {
     "fa_naive_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz,
                           _vp]),
     "fa_diag_exp2": (_i, [_vp, _vp, _vp, _vp, _i, _vp]),
+    "fa_diag_wait_timeout": (_i, [_i, _vp]),
     "fa_get_last_error": (ctypes.c_char_p, []),
     "fa_device_status": (_i, [ctypes.POINTER(ctypes.c_uint)]),
 }
@@ -219,6 +220,11 @@ def diag_exp2(x):
     rc = lib.fa_diag_exp2(_ptr(x), _ptr(y[0]), _ptr(y[1]), _ptr(y[2]), x.numel(), _stream())
     _check(rc, "fa_diag_exp2")
     return tuple(y)
+
+
+def diag_wait_timeout(site: int):
+    """Launch the bounded-wait diagnostic (gives up after ~2 s); read it with device_status()."""
+    _check(load().fa_diag_wait_timeout(int(site), _stream()), "fa_diag_wait_timeout")
 
 
 def device_status() -> int:

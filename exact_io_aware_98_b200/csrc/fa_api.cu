@@ -284,6 +284,12 @@ int fa_diag_exp2(const float* x, float* y_fma, float* y_mufu, float* y_ref, int 
   return check_launch("diag_exp2_kernel");
 }
 
+int fa_diag_wait_timeout(int site, void* stream) {
+  if (site < 1 || site > 0x7fff) return fail(FA_ERR_INVALID, "site must be in [1, 32767]");
+  fa::diag_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(site);
+  return check_launch("diag_wait_timeout_kernel");
+}
+
 size_t fa_naive_workspace_size(int B, int H, int N) {
   if (B < 1 || H < 1 || N < 1) return 0;
   return static_cast<size_t>(B) * H * N * N * 2;

@@ -287,4 +287,19 @@ diag_exp2_kernel(const float* __restrict__ x, float* __restrict__ y_fma, float* 
   }
 }
 
+// Diagnostic: one CTA waits on an mbarrier that nothing ever arrives on, through the same
+// bounded wait the attention kernels use.  The wait gives up after its time limit and records
+// `site` in the status word, which fa_device_status() then reports.  Nothing faults or hangs.
+__global__ void diag_wait_timeout_kernel(int site) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, site);
+}
+
 }  // namespace fa

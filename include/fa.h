@@ -142,6 +142,14 @@ int fa_naive_fwd(const void* q, const void* k, const void* v, void* o, float* ls
  */
 int fa_diag_exp2(const float* x, float* y_fma, float* y_mufu, float* y_ref, int n, void* stream);
 
+/*
+ * fa_diag_wait_timeout -- diagnostic for the device-side failure path: launches one CTA that
+ * waits, through the kernels' bounded mbarrier wait, on a barrier nothing arrives at.  After the
+ * wait's time limit (about 2 s) it records `site` (1..32767) in the status word and returns;
+ * fa_device_status() then reports FA_ERR_TIMEOUT with code (site << 16).  Nothing traps.
+ */
+int fa_diag_wait_timeout(int site, void* stream);
+
 /* Message for the most recent non-OK status returned on this host thread. */
 const char* fa_get_last_error(void);
 

@@ -31,6 +31,10 @@ SMALL = [
     (1, 2, 1100, 128, True, None, True),
     (1, 1, 8, 64, False, None, False),
     (1, 1, 129, 128, True, None, False),
+    (1, 1, 1, 64, True, None, False),
+    (2, 1, 3, 128, False, [2, 3], False),
+    (1, 2, 257, 64, True, [200], True),
+    (2, 1, 390, 128, True, [390, 260], True),
 ]
 
 

@@ -34,6 +34,9 @@ SMALL = [
     (1, 1, 8, 128, True, None, None),
     (1, 2, 129, 64, True, None, None),
     (2, 1, 300, 64, False, [1, 300], None),
+    (1, 1, 3, 128, False, None, None),
+    (2, 2, 650, 64, True, [650, 333], "band"),
+    (1, 1, 255, 128, True, [255], "band"),
 ]
 
 
@@ -138,3 +141,14 @@ def test_tile_reference_and_naive_within_tolerance(cuda_lib):
     torch.cuda.synchronize()
     compare_o(f64(o), o_ref)
     compare_lse(f64(lse), lse_ref, 2e-2)
+
+
+def test_fwd_long_sequence_sampled(cuda_lib):
+    """N = 65536 (B1 H1 d64, causal): 64-bit offsets and 512 KV tiles per head."""
+    x = syn.make_inputs(1, 1, 65536, 64, "bf16", seed=65536, causal=True, with_grad=False)
+    o, lse = run_fwd(cuda_lib, to_gpu(x))
+    rows = np.array([0, 1, 127, 128, 4095, 32767, 32768, 65407, 65408, 65535] +
+                    list(np.random.default_rng(6).choice(65536, 100, replace=False)))
+    o_ref, l_ref = oracle.attn_fwd_rows(x["q"], x["k"], x["v"], x["scale"], rows, True)
+    compare_o(f64(o).reshape(-1, 64)[rows], o_ref)
+    compare_lse(f64(lse).reshape(-1)[rows], l_ref)
