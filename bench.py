@@ -158,6 +158,30 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+# ----------------------------------------------------------------------------- ranks
+def init_distributed(backend: str, timeout_s: int = 120):
+    """One process per GPU (torchrun env); returns torch.distributed or None when WORLD_SIZE=1."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world <= 1:
+        return None
+    import torch.distributed as tdist
+    tdist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return tdist
+
+
+def max_over_ranks(values, dist, device) -> list:
+    """Element-wise max over ranks of per-rank timings (the job is as slow as its slowest rank)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def aggregate_tflops(flop_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput under weak scaling: every rank does one replica's work per step."""
+    return flop_per_rank_step * world / (ms_per_step * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------- our arm
 def run_ours(args, rank: int, world: int, dist):
     import exact_io_aware_98_b200 as fa
@@ -206,10 +230,7 @@ def run_ours(args, rank: int, world: int, dist):
     total_ms = ev[0][0].elapsed_time(ev[K - 1][2])
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
-    t = torch.tensor([total_ms, fwd_ms, bwd_ms], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, fwd_ms, bwd_ms = (float(v) for v in t.tolist())
+    total_ms, fwd_ms, bwd_ms = max_over_ranks([total_ms, fwd_ms, bwd_ms], dist, dev)
     status = fa.device_status()
 
     # ---- end to end through the public API: pinned host inputs in, results back to host
@@ -246,16 +267,13 @@ def run_ours(args, rank: int, world: int, dist):
             e2e_step()
         e1.record()
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if dist is not None:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        ms_e = float(te.item()) / Ke
-        e2e = {"value": round((f_fwd + f_bwd) * world / (ms_e * 1e-3) / 1e12, 3),
+        ms_e = max_over_ranks([e0.elapsed_time(e1)], dist, dev)[0] / Ke
+        e2e = {"value": round(aggregate_tflops(f_fwd + f_bwd, world, ms_e), 3),
                "unit": "TFLOP/s", "ms_per_step": round(ms_e, 4), "steps": Ke,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     ms_step = total_ms / K
-    value = (f_fwd + f_bwd) * world / (ms_step * 1e-3) / 1e12
+    value = aggregate_tflops(f_fwd + f_bwd, world, ms_step)
     peaks, peak_src = load_peaks()
     sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -409,12 +427,9 @@ def main():
         if rank == 0:
             print(json.dumps(run_reference(args, world)), flush=True)
         return
-    dist = None
     if world > 1:
-        import torch.distributed as tdist
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
-        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-        dist = tdist
+    dist = init_distributed("nccl")
     try:
         line, (x, g, o, lse, dq) = run_ours(args, rank, world, dist)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
