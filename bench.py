@@ -367,9 +367,15 @@ def deviation_sweep():
     kw = dict(scale=g["scale"], kv_len=g["kv_len"])
     o_tc, _ = fa.fwd(g["q"], g["k"], g["v"], **kw)
     out["tcgen05_Br128_Bc128_lazy"] = stat(o_tc)
+    # the study's axes: key-tile width Bc, the order the key tiles are visited in, and whether
+    # the normaliser l sums the fp32 P or the bf16-rounded P that enters P.V
     for bc in (64, 128, 256):
-        o_t, _ = fa.fwd_tile_reference(g["q"], g["k"], g["v"], bc, **kw)
-        out[f"tile_Bc{bc}"] = stat(o_t)
+        for reverse in (False, True):
+            for l_rounded in (False, True):
+                o_t, _ = fa.fwd_tile_reference(g["q"], g["k"], g["v"], bc, reverse=reverse,
+                                               l_rounded=l_rounded, **kw)
+                key = f"tile_Bc{bc}_{'reverse' if reverse else 'forward'}_l{'bf16' if l_rounded else 'fp32'}"
+                out[key] = stat(o_t)
     o_n, _ = fa.naive_fwd(g["q"], g["k"], g["v"], **kw)
     out["naive_materialised"] = stat(o_n)
     diff = (o_tc.float() - o_n.float()).abs()

@@ -31,7 +31,7 @@ SIGNATURES = {
     "fa_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
                             _vp, _vp, _i, _vp]),
     "fa_fwd_tile_reference": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp,
-                                   _i, _vp]),
+                                   _i, _i, _vp]),
     "fa_naive_workspace_size": (_sz, [_i, _i, _i]),
     "fa_naive_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _sz,
                           _vp]),
@@ -176,9 +176,15 @@ def bwd_noalloc(q, k, v, o, lse, do, scale: Optional[float] = None, causal: bool
     return dq, dk, dv
 
 
+TILE_REVERSE = 1     # fa.h FA_TILE_REVERSE: key tiles visited last to first
+TILE_L_ROUNDED = 2   # fa.h FA_TILE_L_ROUNDED: l sums the bf16-rounded P
+
+
 def fwd_tile_reference(q, k, v, bc: int, scale: Optional[float] = None, causal: bool = False,
-                       block_mask=None, kv_len=None):
-    """bf16 CUDA-core forward that rescales after every `bc` keys (deviation study)."""
+                       block_mask=None, kv_len=None, reverse: bool = False,
+                       l_rounded: bool = False):
+    """bf16 CUDA-core forward that rescales after every `bc` keys (deviation study); `reverse`
+    visits the key tiles last to first, `l_rounded` sums l over the bf16-rounded P."""
     lib = load()
     B, H, N, d = q.shape
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -188,7 +194,9 @@ def fwd_tile_reference(q, k, v, bc: int, scale: Optional[float] = None, causal: 
     bm, kl = _masks(block_mask, kv_len)
     s = default_scale(d) if scale is None else float(scale)
     rc = lib.fa_fwd_tile_reference(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, H, N, d, s,
-                                   int(causal), bm, kl, int(bc), _stream())
+                                   int(causal), bm, kl, int(bc),
+                                   (TILE_REVERSE if reverse else 0) |
+                                   (TILE_L_ROUNDED if l_rounded else 0), _stream())
     _check(rc, "fa_fwd_tile_reference")
     return o, l
 

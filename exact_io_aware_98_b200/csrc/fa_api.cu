@@ -209,7 +209,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
     const long long rows = static_cast<long long>(B) * H * N;
     fa::fa_fwd_rowwarp_kernel<float, false><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
         static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-        static_cast<float*>(o), lse, block_mask, kv_len, B, H, N, d, scale, causal ? 1 : 0, 128);
+        static_cast<float*>(o), lse, block_mask, kv_len, B, H, N, d, scale, causal ? 1 : 0, 128, 0);
     return check_launch("fa_fwd_rowwarp_kernel<f32>");
   }
   return fail(FA_ERR_INVALID, "unknown dtype %d", dtype);
@@ -261,18 +261,20 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
 
 int fa_fwd_tile_reference(const void* q, const void* k, const void* v, void* o, float* lse,
                           int B, int H, int N, int d, float scale, int causal,
-                          const uint8_t* block_mask, const int32_t* kv_len, int bc,
+                          const uint8_t* block_mask, const int32_t* kv_len, int bc, int flags,
                           void* stream) {
   int rc = common_checks(q, k, v, o, lse, B, H, N, d, scale);
   if (rc != FA_OK) return rc;
   if (d > 128) return fail(FA_ERR_UNSUPPORTED, "d <= 128 required, got %d", d);
   if (bc < 32 || bc > 256 || (bc % 32) != 0) return fail(FA_ERR_INVALID, "bc must be 32..256 in steps of 32");
+  if ((flags & ~(FA_TILE_REVERSE | FA_TILE_L_ROUNDED)) != 0)
+    return fail(FA_ERR_INVALID, "unknown tile-reference flags 0x%x", flags);
   const long long rows = static_cast<long long>(B) * H * N;
   fa::fa_fwd_rowwarp_kernel<__nv_bfloat16, true>
       <<<static_cast<unsigned>((rows + 7) / 8), 256, 0, static_cast<cudaStream_t>(stream)>>>(
           static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
           static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), lse, block_mask,
-          kv_len, B, H, N, d, scale, causal ? 1 : 0, bc);
+          kv_len, B, H, N, d, scale, causal ? 1 : 0, bc, flags);
   return check_launch("fa_fwd_rowwarp_kernel<bf16>");
 }
 

@@ -146,8 +146,12 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       return false;
     return true;
   };
+  // steps of this CTA: a closed form unless a block mask decides tile by tile (a loop over all
+  // query tiles in every thread costs thousands of cycles per CTA at N = 16384)
+  const int it_first = p.causal ? k0 / BM : 0;  // query tiles before it_first see no key here
   int n_steps = 0;
-  for (int it = 0; it < n_qt; ++it) n_steps += q_active(it) ? 1 : 0;
+  if (p.block_mask == nullptr) n_steps = kv_live ? n_qt - it_first : 0;
+  else for (int it = it_first; it < n_qt; ++it) n_steps += q_active(it) ? 1 : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv, 1);
@@ -190,7 +194,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         tma_load_3d(smem + L::OFF_V + s * L::KV_SUBTILE, &tm_v, bar_kv, s * 64, k0, bh);
       }
       int t = 0;
-      for (int it = 0; it < n_qt; ++it) {
+      for (int it = it_first; it < n_qt; ++it) {
         if (!q_active(it)) continue;
         const int st = t % L::QST;
         if (t >= L::QST &&
@@ -348,7 +352,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     const float scale2 = p.scale2;
     bool ok = true;
     int t = 0;
-    for (int it = 0; it < n_qt; ++it) {
+    for (int it = it_first; it < n_qt; ++it) {
       if (!q_active(it)) continue;
       const int st = t % L::QST;
       const int buf = t & 1;
@@ -508,7 +512,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int qw = warp & 3;
     const uint32_t t_lane = static_cast<uint32_t>(32 * qw) << 16;
     int t = 0;
-    for (int it = 0; it < n_qt; ++it) {
+    for (int it = it_first; it < n_qt; ++it) {
       if (!q_active(it)) continue;
       const int buf = t & 1;
       const int i0 = it * BM;

@@ -5,7 +5,10 @@
 //         article calls out under "fp16/bf16 support"), and
 //       - the tile-width reference for the numeric-deviation sweep of "Is Flash Attention
 //         Stable?" (aibr.jp summary, section 3): bf16 inputs, the running maximum is updated
-//         at every Bc-key tile (no lazy threshold) and P is rounded to bf16 before P.V.
+//         at every Bc-key tile (no lazy threshold) and P is rounded to bf16 before P.V.  Two
+//         more axes of that study are flags: the order in which the key tiles are visited
+//         (first to last, or last to first), and whether the normaliser l sums the fp32 P or
+//         the bf16-rounded P that enters P.V.
 //   * naive_* kernels: the materialised "Baseline Attention" of the same study -- S written to
 //     HBM in bf16, row softmax from it with P written back in bf16, then P.V.
 //   * bwd_preprocess_kernel / dq_convert_kernel: the elementwise steps around the tensor-core
@@ -40,12 +43,16 @@ __device__ __forceinline__ bool key_allowed(int i, int j, int kvlen, int causal,
 
 // One warp per query row.  Keys are processed in tiles of `bc` (a multiple of 32, <= 256);
 // lane l holds the scores of keys tile0 + 32*u + l.  Output column c = 32*u + lane.
+// flags: kTileReverse visits the key tiles last to first; kTileLRounded sums l over the
+// rounded P (only meaningful with ROUND_P).
+constexpr int kTileReverse = 1;
+constexpr int kTileLRounded = 2;
 template <typename T, bool ROUND_P>
 __global__ void __launch_bounds__(256)
 fa_fwd_rowwarp_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                       T* __restrict__ o, float* __restrict__ lse, const uint8_t* block_mask,
                       const int32_t* kv_len, int B, int H, int N, int d, float scale, int causal,
-                      int bc) {
+                      int bc, int flags) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row_g = static_cast<long long>(blockIdx.x) * 8 + warp;  // flat bh*N + i
   if (row_g >= static_cast<long long>(B) * H * N) return;
@@ -61,7 +68,10 @@ fa_fwd_rowwarp_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
   const int ncol = (d + 31) / 32;  // <= 4
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   float m = -INFINITY, l = 0.f;
-  for (int t0 = 0; t0 < N; t0 += bc) {
+  const int n_tiles = (N + bc - 1) / bc;
+  const bool l_rounded = ROUND_P && (flags & kTileLRounded) != 0;
+  for (int tt = 0; tt < n_tiles; ++tt) {
+    const int t0 = ((flags & kTileReverse) ? n_tiles - 1 - tt : tt) * bc;
     float sc[8];
     float tmax = -INFINITY;
 #pragma unroll
@@ -85,8 +95,9 @@ fa_fwd_rowwarp_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const float pe = (sc[u] == -INFINITY) ? 0.f : expf(sc[u] - m_new);
-      psum += pe;
-      sc[u] = ROUND_P ? __bfloat162float(__float2bfloat16_rn(pe)) : pe;
+      const float pr = ROUND_P ? __bfloat162float(__float2bfloat16_rn(pe)) : pe;
+      psum += l_rounded ? pr : pe;
+      sc[u] = pr;
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);

@@ -108,16 +108,24 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                    float scale, int causal, const uint8_t* block_mask, const int32_t* kv_len,
                    int dtype, void* stream);
 
+/* Flags of fa_fwd_tile_reference: the other two axes of the deviation study. */
+enum {
+  FA_TILE_REVERSE = 1,    /* visit the key tiles from the last to the first */
+  FA_TILE_L_ROUNDED = 2   /* the normaliser l sums the bf16-rounded P that enters P.V (else the
+                             fp32 P before rounding) */
+};
+
 /*
- * fa_fwd_tile_reference -- bf16 forward on CUDA cores for the tile-size numeric-deviation
- * study of "Is Flash Attention Stable?" (aibr.jp summary, sections 3-4): the running maximum
- * and sum are rescaled after every tile of `bc` keys (bc in {32, 64, ..., 256}) and P is
- * rounded to bf16 before P.V, as in a tensor-core kernel with that key-tile width.  Same
+ * fa_fwd_tile_reference -- bf16 forward on CUDA cores for the numeric-deviation study of "Is
+ * Flash Attention Stable?" (aibr.jp summary, sections 3-4): the running maximum and sum are
+ * rescaled after every tile of `bc` keys (bc in {32, 64, ..., 256}) and P is rounded to bf16
+ * before P.V, as in a tensor-core kernel with that key-tile width.  `flags` (FA_TILE_*) picks
+ * the tile order and which P the normaliser sums; unknown bits give FA_ERR_INVALID.  Same
  * layouts, masks and errors as fa_fwd (bf16, 1 <= d <= 128).  Not a fast path.
  */
 int fa_fwd_tile_reference(const void* q, const void* k, const void* v, void* o, float* lse,
                           int B, int H, int N, int d, float scale, int causal,
-                          const uint8_t* block_mask, const int32_t* kv_len, int bc,
+                          const uint8_t* block_mask, const int32_t* kv_len, int bc, int flags,
                           void* stream);
 
 /* Bytes of workspace fa_naive_fwd needs: the materialised S / P matrix, [B][H][N][N] bf16. */

@@ -36,6 +36,12 @@ def test_header_declares_the_boundary():
         assert required in names
 
 
+def test_binding_constants_match_header():
+    text = open(HEADER).read()
+    vals = {k: int(v) for k, v in re.findall(r"\b(FA_TILE_[A-Z_]+)\s*=\s*(\d+)", text)}
+    assert vals == {"FA_TILE_REVERSE": fa.TILE_REVERSE, "FA_TILE_L_ROUNDED": fa.TILE_L_ROUNDED}
+
+
 def test_every_declared_symbol_is_exported(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
@@ -88,10 +94,13 @@ def test_bwd_validation_codes(lib):
 
 
 def test_aux_entry_validation(lib):
-    assert lib.fa_fwd_tile_reference(A, A, A, A, A, 1, 1, 64, 64, 0.125, 0, None, None, 48,
+    assert lib.fa_fwd_tile_reference(A, A, A, A, A, 1, 1, 64, 64, 0.125, 0, None, None, 48, 0,
                                      None) == INVALID
-    assert lib.fa_fwd_tile_reference(A, A, A, A, A, 1, 1, 64, 192, 0.125, 0, None, None, 64,
+    assert lib.fa_fwd_tile_reference(A, A, A, A, A, 1, 1, 64, 192, 0.125, 0, None, None, 64, 0,
                                      None) == UNSUPPORTED
+    assert lib.fa_fwd_tile_reference(A, A, A, A, A, 1, 1, 64, 64, 0.125, 0, None, None, 64, 4,
+                                     None) == INVALID
+    assert "flags" in lib.fa_get_last_error().decode()
     assert lib.fa_naive_fwd(A, A, A, A, A, 1, 1, 64, 64, 0.125, 0, None, None, A, 16,
                             None) == WORKSPACE
 

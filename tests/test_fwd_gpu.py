@@ -143,6 +143,35 @@ def test_tile_reference_and_naive_within_tolerance(cuda_lib):
     compare_lse(f64(lse), lse_ref, 2e-2)
 
 
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("l_rounded", [False, True])
+def test_tile_reference_deviation_axes(cuda_lib, reverse, l_rounded):
+    """Both tile orders and both normalisers of the deviation study stay within tolerance.  The
+    normaliser over rounded P changes l by a relative 2^-9 at most (bf16's rounding of P), which
+    moves lse by at most -log(1 - 2^-9) on top of the usual 1e-3."""
+    x = syn.make_inputs(2, 2, 520, 64, "bf16", seed=13, causal=True, with_grad=False)
+    g = to_gpu(x)
+    o_ref, lse_ref = oracle_fwd(x)
+    for bc in (64, 256):
+        o, lse = cuda_lib.fwd_tile_reference(g["q"], g["k"], g["v"], bc, g["scale"], True,
+                                             reverse=reverse, l_rounded=l_rounded)
+        torch.cuda.synchronize()
+        compare_o(f64(o), o_ref)
+        compare_lse(f64(lse), lse_ref, 1e-3 - (np.log1p(-2.0 ** -9) if l_rounded else 0.0))
+
+
+def test_tile_reference_rounded_normaliser_rows_sum_to_one(cuda_lib):
+    """l over the rounded P that multiplies V: V = 1 gives O = 1 exactly after bf16 rounding."""
+    x = syn.make_inputs(1, 2, 300, 64, "bf16", seed=14, causal=True, with_grad=False)
+    g = to_gpu(x)
+    ones = torch.ones_like(g["v"])
+    for reverse in (False, True):
+        o, _ = cuda_lib.fwd_tile_reference(g["q"], g["k"], ones, 64, g["scale"], True,
+                                           reverse=reverse, l_rounded=True)
+        torch.cuda.synchronize()
+        assert torch.all(o == 1)
+
+
 def test_fwd_long_sequence_sampled(cuda_lib):
     """N = 65536 (B1 H1 d64, causal): 64-bit offsets and 512 KV tiles per head."""
     x = syn.make_inputs(1, 1, 65536, 64, "bf16", seed=65536, causal=True, with_grad=False)

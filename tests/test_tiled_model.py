@@ -63,3 +63,54 @@ def test_bf16_p_rounding_stays_inside_tolerance():
                               round_p_bf16=True, dtype=np.float32)
     err = np.abs(o - o_ref[0, 0])
     assert err.max() < 2e-2 and err.mean() < 2e-3
+
+
+@pytest.mark.parametrize("Bc", [64, 128, 256])
+@pytest.mark.parametrize("mask", ["none", "causal", "padding"])
+def test_reverse_tile_order_is_exact(Bc, mask):
+    """Visiting the key tiles last to first changes nothing in exact arithmetic: the tile-order
+    axis of "Is Flash Attention Stable?" (aibr.jp summary, section 3) only moves rounding."""
+    N, d = 333, 16
+    q, k, v = (R.standard_normal((N, d)) * a for a in (2.0, 2.0, 1.0))
+    causal = mask == "causal"
+    L = 250 if mask == "padding" else None
+    o_ref, lse_ref = oracle.attn_fwd(q[None, None], k[None, None], v[None, None], 0.25, causal,
+                                     None, None if L is None else np.array([L]))
+    for lazy in (0.0, 8.0):
+        o, lse = tiled_forward_head(q, k, v, 0.25, causal, L, Bc=Bc, lazy_threshold=lazy,
+                                    reverse=True)
+        assert np.max(np.abs(o - o_ref[0, 0])) < 1e-12
+        assert np.max(np.abs(lse - lse_ref[0, 0])) < 1e-12
+
+
+def test_rounded_normaliser_makes_rows_sum_to_one():
+    """With l summed over the same bf16-rounded P that multiplies V, the effective attention
+    weights of a row sum to one: V = 1 gives O = 1 to fp64 rounding.  With l over the unrounded
+    P the ratio sum(round(P)) / sum(P) is left in O (reading c-7 of the normaliser choice)."""
+    N, d = 256, 8
+    q, k = (R.standard_normal((N, d)) * 2.0 for _ in range(2))
+    v = np.ones((N, 4))
+    o_r, _ = tiled_forward_head(q, k, v, 0.35, True, Bc=64, round_p_bf16=True, l_rounded=True)
+    assert np.max(np.abs(o_r - 1.0)) < 1e-13
+    o_f, _ = tiled_forward_head(q, k, v, 0.35, True, Bc=64, round_p_bf16=True, l_rounded=False)
+    dev = np.abs(o_f - 1.0)
+    assert dev.max() > 1e-6            # the rounding of P shows
+    assert dev.max() < 2.0 ** -8       # but stays within bf16's relative rounding of P
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("l_rounded", [False, True])
+def test_deviation_axes_stay_inside_tolerance(reverse, l_rounded):
+    """fp32 arithmetic, bf16 P, both tile orders and both normalisers, on the long-context value
+    scale: every variant of the deviation sweep stays within the bf16 tolerance of the oracle."""
+    N, d = 512, 64
+    torch = __import__("torch")
+    q, k = (R.standard_normal((N, d)) * 2.0 for _ in range(2))
+    v = R.standard_normal((N, d))
+    qb, kb, vb = (torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).float().numpy()
+                  for x in (q, k, v))
+    o_ref, _ = oracle.attn_fwd(qb[None, None], kb[None, None], vb[None, None], 0.125, True)
+    o, _ = tiled_forward_head(qb, kb, vb, 0.125, True, Bc=64, round_p_bf16=True,
+                              dtype=np.float32, reverse=reverse, l_rounded=l_rounded)
+    err = np.abs(o - o_ref[0, 0])
+    assert err.max() < 2e-2 and err.mean() < 2e-3

@@ -13,7 +13,11 @@ Options mirror the kernel's choices:
     maximum exceeds it by more than this many log2 units (0 = always).
     The final division by l uses the same reference, so the result is exact.
   * ``round_p_bf16``: round P to bfloat16 before the P.V product (the tensor
-    core consumes bf16 P); l is summed from the unrounded fp32-or-fp64 P.
+    core consumes bf16 P); l is summed from the unrounded fp32-or-fp64 P unless
+    ``l_rounded`` is set, in which case l sums the rounded P that enters P.V.
+  * ``reverse``: visit the key tiles from the last to the first.  In exact
+    arithmetic the order does not matter; in floating point it is one of the
+    axes of the deviation study in "Is Flash Attention Stable?".
   * ``dtype``: float64 (exactness check) or float32 (kernel-like arithmetic).
 """
 from __future__ import annotations
@@ -31,7 +35,7 @@ def _bf16(x: np.ndarray) -> np.ndarray:
 
 def tiled_forward_head(q, k, v, scale, causal=False, L=None, block_mask=None, block=128,
                        Br=128, Bc=128, lazy_threshold=0.0, round_p_bf16=False,
-                       dtype=np.float64):
+                       dtype=np.float64, reverse=False, l_rounded=False):
     q = np.asarray(q, dtype)
     k = np.asarray(k, dtype)
     v = np.asarray(v, dtype)
@@ -45,7 +49,8 @@ def tiled_forward_head(q, k, v, scale, causal=False, L=None, block_mask=None, bl
         m = np.full(len(rows), -np.inf, dtype)
         l = np.zeros(len(rows), dtype)
         acc = np.zeros((len(rows), v.shape[1]), dtype)
-        for c0 in range(0, N, Bc):
+        starts = list(range(0, N, Bc))
+        for c0 in (starts[::-1] if reverse else starts):
             cols = np.arange(c0, min(c0 + Bc, N))
             allowed = (cols[None, :] < L) & np.ones((len(rows), 1), bool)
             if causal:
@@ -68,8 +73,8 @@ def tiled_forward_head(q, k, v, scale, causal=False, L=None, block_mask=None, bl
             base = np.where(np.isneginf(m_new), 0.0, m_new)
             p = np.exp2(s - base[:, None]).astype(dtype)
             p = np.where(allowed, p, 0.0).astype(dtype)
-            l = alpha * l + p.sum(axis=1, dtype=dtype)
             pv = _bf16(p) if round_p_bf16 else p
+            l = alpha * l + (pv if l_rounded else p).sum(axis=1, dtype=dtype)
             acc = alpha[:, None] * acc + (pv @ v[cols]).astype(dtype)
             m = m_new
         ok = l > 0
