@@ -179,6 +179,45 @@ def attn_bwd_dq_rows(q, k, v, do, scale: float, rows: Sequence[int], causal: boo
     return dq
 
 
+def kv_group(H: int, H_kv: int) -> int:
+    """Query heads per K/V head; H must be a multiple of H_kv."""
+    if H_kv < 1 or H % H_kv != 0:
+        raise ValueError(f"H = {H} is not a multiple of H_kv = {H_kv}")
+    return H // H_kv
+
+
+def attn_fwd_gqa(q, k, v, scale: float, causal: bool = False, block_mask=None, kv_len=None,
+                 block: int = 128):
+    """Grouped-query attention, the MQA/GQA of the tcdigital FA-2 ROI article (section
+    "MQA/GQA ... との相乗効果"): q is [B,H,N,d], k and v are [B,H_kv,N,d], and query head h
+    reads K/V head h // (H / H_kv) (contiguous groups; H_kv = 1 is multi-query attention).
+    Written as the definition: ordinary attention with every K/V head repeated for the query
+    heads of its group."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    G = kv_group(q.shape[1], k.shape[1])
+    return attn_fwd(q, np.repeat(k, G, axis=1), np.repeat(v, G, axis=1), scale, causal,
+                    block_mask, kv_len, block)
+
+
+def attn_bwd_gqa(q, k, v, do, scale: float, causal: bool = False, block_mask=None,
+                 kv_len=None, block: int = 128, kv_heads: Optional[Sequence[int]] = None):
+    """dQ [B,H,N,d] and dK, dV [B,H_kv,N,d] of grouped-query attention.  A K/V head enters the
+    output of every query head of its group, so by the chain rule through the repetition its
+    gradient is the sum of the per-query-head gradients.  With ``kv_heads`` (flat b*H_kv + j)
+    only those K/V heads and the query heads of their groups are filled."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, H, N, d = q.shape
+    H_kv = k.shape[1]
+    G = kv_group(H, H_kv)
+    heads = None
+    if kv_heads is not None:
+        heads = [(j // H_kv) * H + (j % H_kv) * G + g for j in kv_heads for g in range(G)]
+    dq, dk, dv = attn_bwd(q, np.repeat(k, G, axis=1), np.repeat(v, G, axis=1), do, scale,
+                          causal, block_mask, kv_len, block, heads)
+    return (dq, dk.reshape(B, H_kv, G, N, d).sum(axis=2),
+            dv.reshape(B, H_kv, G, N, d).sum(axis=2))
+
+
 def attn_probs(q, k, scale: float, causal: bool = False, block_mask=None, kv_len_b: int = -1,
                block: int = 128):
     """A (N x N) and lse (N) of one head; q, k are [N, d]."""

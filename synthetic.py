@@ -117,15 +117,18 @@ def make_inputs(B: int, H: int, N: int, d: int, dtype: str = "bf16", seed: int =
                 qk_amp: float = 1.0, causal: bool = False,
                 kv_len: Optional[np.ndarray] = None,
                 block_mask: Optional[np.ndarray] = None,
-                with_grad: bool = True) -> dict:
-    """Seeded CPU tensors in [B, H, N, d] layout (contiguous)."""
+                with_grad: bool = True, H_kv: Optional[int] = None) -> dict:
+    """Seeded CPU tensors in [B, H, N, d] layout (contiguous).  With ``H_kv`` (grouped-query
+    attention) K and V are [B, H_kv, N, d]."""
     shape = (B, H, N, d)
+    kv_shape = shape if H_kv is None else (B, H_kv, N, d)
     out = {
         "B": B, "H": H, "N": N, "d": d, "dtype": dtype, "seed": seed,
+        "H_kv": H if H_kv is None else H_kv,
         "scale": scale_for(d), "causal": bool(causal),
         "q": _to_dtype(_normal(seed + T_Q, shape, qk_amp), dtype),
-        "k": _to_dtype(_normal(seed + T_K, shape, qk_amp), dtype),
-        "v": _to_dtype(_normal(seed + T_V, shape, 1.0), dtype),
+        "k": _to_dtype(_normal(seed + T_K, kv_shape, qk_amp), dtype),
+        "v": _to_dtype(_normal(seed + T_V, kv_shape, 1.0), dtype),
         "kv_len": None if kv_len is None else torch.from_numpy(np.asarray(kv_len, np.int32)),
         "block_mask": None if block_mask is None else torch.from_numpy(
             np.ascontiguousarray(block_mask, dtype=np.uint8)),
