@@ -385,6 +385,39 @@ def deviation_sweep():
     return out
 
 
+def gqa_measurement(iters: int = 10):
+    """Grouped-query attention (the MQA/GQA of the tcdigital FA-2 ROI article) on a Llama-class
+    grouping: B1 H32 H_kv8 N8192 d128 causal.  FLOPs count per query head, as for attention with
+    H heads; the K/V reads shrink by H/H_kv."""
+    import exact_io_aware_98_b200 as fa
+    B, H, H_kv, N, d = 1, 32, 8, 8192, 128
+    x = syn.make_inputs(B, H, N, d, "bf16", seed=1400, qk_amp=2.0, causal=True, H_kv=H_kv)
+    g = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
+    f_fwd, f_bwd = flops(x, H)
+    o = torch.empty_like(g["q"])
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    dq, dk, dv = torch.empty_like(g["q"]), torch.empty_like(g["k"]), torch.empty_like(g["v"])
+    ws = torch.empty(fa.bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
+    kw = dict(scale=g["scale"], causal=True)
+    for _ in range(3):
+        fa.fwd(g["q"], g["k"], g["v"], out=o, lse=lse, **kw)
+        fa.bwd(g["q"], g["k"], g["v"], o, lse, g["do"], workspace=ws, dq=dq, dk=dk, dv=dv, **kw)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record()
+    for _ in range(iters):
+        fa.fwd(g["q"], g["k"], g["v"], out=o, lse=lse, **kw)
+    ev[1].record()
+    for _ in range(iters):
+        fa.bwd(g["q"], g["k"], g["v"], o, lse, g["do"], workspace=ws, dq=dq, dk=dk, dv=dv, **kw)
+    ev[2].record()
+    torch.cuda.synchronize()
+    fwd_ms, bwd_ms = ev[0].elapsed_time(ev[1]) / iters, ev[1].elapsed_time(ev[2]) / iters
+    return {"config": f"B{B} H{H} H_kv{H_kv} N{N} d{d} causal, bf16 (Q,K x2)",
+            "fwd": {"ms": round(fwd_ms, 4), "tflops": round(f_fwd / fwd_ms / 1e9, 2)},
+            "bwd": {"ms": round(bwd_ms, 4), "tflops": round(f_bwd / bwd_ms / 1e9, 2)},
+            "device_status": fa.device_status()}
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args, world: int):
     import oracle
@@ -443,6 +476,7 @@ def main():
             line["cpu_baseline"] = cpu
             line["max_err_vs_fp64"] = err
             line["deviation_sweep"] = deviation_sweep()
+            line["gqa"] = gqa_measurement()
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

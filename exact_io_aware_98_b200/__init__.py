@@ -25,7 +25,10 @@ _STATUS = {0: "FA_OK", -1: "FA_ERR_INVALID", -2: "FA_ERR_UNSUPPORTED", -3: "FA_E
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "fa_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp, _i, _vp]),
+    "fa_fwd_gqa": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _vp, _vp, _i, _vp]),
     "fa_bwd_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "fa_bwd_gqa": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i,
+                        _vp, _vp, _i, _vp, _sz, _vp]),
     "fa_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp,
                     _vp, _i, _vp, _sz, _vp]),
     "fa_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
@@ -107,24 +110,42 @@ def default_scale(d: int) -> float:
     return float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32).item())
 
 
+def _kv_heads(q, k, v) -> int:
+    """K/V head count; k and v are [B, H_kv, N, d] with H a multiple of H_kv."""
+    B, H, N, d = q.shape
+    H_kv = k.shape[1]
+    for t, n in ((k, "k"), (v, "v")):
+        if t.dim() != 4 or (t.shape[0], t.shape[2], t.shape[3]) != (B, N, d) or t.shape[1] != H_kv:
+            raise FaError(f"{n} shape {tuple(t.shape)} does not match q {tuple(q.shape)}")
+    if H_kv < 1 or H % H_kv != 0:
+        raise FaError(f"H = {H} is not a multiple of H_kv = {H_kv}")
+    return H_kv
+
+
 def fwd(q, k, v, scale: Optional[float] = None, causal: bool = False, block_mask=None,
         kv_len=None, out=None, lse=None):
-    """O, lse = fa_fwd(q, k, v); tensors [B, H, N, d] (bf16 or fp32) on the GPU."""
+    """O, lse = fa_fwd(q, k, v); q [B, H, N, d], k and v [B, H_kv, N, d] (bf16 or fp32) on the
+    GPU.  H_kv < H is grouped-query attention (fa_fwd_gqa): query head h reads K/V head
+    h // (H / H_kv)."""
     lib = load()
     B, H, N, d = q.shape
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _require(t, n, q.dtype)
-        if t.shape != q.shape:
-            raise FaError(f"{n} shape {tuple(t.shape)} != q shape {tuple(q.shape)}")
+    H_kv = _kv_heads(q, k, v)
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
     _require(o, "out", q.dtype)
     _require(l, "lse", torch.float32)
     bm, kl = _masks(block_mask, kv_len)
     s = default_scale(d) if scale is None else float(scale)
-    rc = lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, H, N, d, s, int(causal),
-                    bm, kl, _dtype_code(q), _stream())
-    _check(rc, "fa_fwd")
+    if H_kv == H:
+        rc = lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, H, N, d, s, int(causal),
+                        bm, kl, _dtype_code(q), _stream())
+        _check(rc, "fa_fwd")
+    else:
+        rc = lib.fa_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, H, H_kv, N, d, s,
+                            int(causal), bm, kl, _dtype_code(q), _stream())
+        _check(rc, "fa_fwd_gqa")
     return o, l
 
 
@@ -134,24 +155,36 @@ def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
 
 def bwd(q, k, v, o, lse, do, scale: Optional[float] = None, causal: bool = False,
         block_mask=None, kv_len=None, workspace=None, dq=None, dk=None, dv=None):
-    """dQ, dK, dV = fa_bwd(...); bf16 tensors [B, H, N, d] on the GPU."""
+    """dQ, dK, dV = fa_bwd(...); bf16 tensors on the GPU, q/o/do [B, H, N, d], k/v and dK/dV
+    [B, H_kv, N, d] (fa_bwd_gqa when H_kv < H)."""
     lib = load()
     B, H, N, d = q.shape
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
         _require(t, n, q.dtype)
+    H_kv = _kv_heads(q, k, v)
     _require(lse, "lse", torch.float32)
     need = bwd_workspace_size(B, H, N, d)
     ws = torch.empty(need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
     _require(ws, "workspace", torch.uint8)
     dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _require(t, n, q.dtype)
+    if dq.shape != q.shape or dk.shape != k.shape or dv.shape != v.shape:
+        raise FaError("gradient shapes must match q, k and v")
     bm, kl = _masks(block_mask, kv_len)
     s = default_scale(d) if scale is None else float(scale)
-    rc = lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
-                    _ptr(dv), B, H, N, d, s, int(causal), bm, kl, _dtype_code(q), _ptr(ws),
-                    ws.numel(), _stream())
-    _check(rc, "fa_bwd")
+    if H_kv == H:
+        rc = lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq),
+                        _ptr(dk), _ptr(dv), B, H, N, d, s, int(causal), bm, kl, _dtype_code(q),
+                        _ptr(ws), ws.numel(), _stream())
+        _check(rc, "fa_bwd")
+    else:
+        rc = lib.fa_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq),
+                            _ptr(dk), _ptr(dv), B, H, H_kv, N, d, s, int(causal), bm, kl,
+                            _dtype_code(q), _ptr(ws), ws.numel(), _stream())
+        _check(rc, "fa_bwd_gqa")
     return dq, dk, dv
 
 

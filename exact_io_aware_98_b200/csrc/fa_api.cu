@@ -113,15 +113,15 @@ BwdWs bwd_ws(int B, int H, int N, int d) {
 
 template <int D>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-               int N, float scale, int causal, const uint8_t* bm, const int32_t* kv_len,
-               cudaStream_t stream) {
+               int H_kv, int N, float scale, int causal, const uint8_t* bm,
+               const int32_t* kv_len, cudaStream_t stream) {
   using L = fa::FwdLayout<D>;
   CUtensorMap mq, mk, mv;
   const int BH = B * H;
   int rc;
   if ((rc = make_map(&mq, q, BH, N, D, 128, "q")) != FA_OK) return rc;
-  if ((rc = make_map(&mk, k, BH, N, D, 128, "k")) != FA_OK) return rc;
-  if ((rc = make_map(&mv, v, BH, N, D, 128, "v")) != FA_OK) return rc;
+  if ((rc = make_map(&mk, k, B * H_kv, N, D, 128, "k")) != FA_OK) return rc;
+  if ((rc = make_map(&mv, v, B * H_kv, N, D, 128, "v")) != FA_OK) return rc;
   if ((rc = set_smem(fa::fa_fwd_sm100_kernel<D>, L::SMEM_ALLOC)) != FA_OK) return rc;
   fa::FwdParams p;
   p.block_mask = bm;
@@ -130,6 +130,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.lse = lse;
   p.B = B;
   p.H = H;
+  p.H_kv = H_kv;
   p.N = N;
   p.n_mtiles = (N + 255) / 256;
   p.scale2 = scale * kLog2e;
@@ -142,15 +143,15 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 
 template <int D>
 int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
-               int B, int H, int N, float scale, int causal, const uint8_t* bm,
+               int B, int H, int H_kv, int N, float scale, int causal, const uint8_t* bm,
                const int32_t* kv_len, const BwdWs& ws, uint8_t* wsb, cudaStream_t stream) {
   using L = fa::BwdLayout<D>;
   CUtensorMap mq, mk, mv, mdo;
   const int BH = B * H;
   int rc;
   if ((rc = make_map(&mq, q, BH, N, D, L::BM, "q")) != FA_OK) return rc;
-  if ((rc = make_map(&mk, k, BH, N, D, 128, "k")) != FA_OK) return rc;
-  if ((rc = make_map(&mv, v, BH, N, D, 128, "v")) != FA_OK) return rc;
+  if ((rc = make_map(&mk, k, B * H_kv, N, D, 128, "k")) != FA_OK) return rc;
+  if ((rc = make_map(&mv, v, B * H_kv, N, D, 128, "v")) != FA_OK) return rc;
   if ((rc = make_map(&mdo, dO, BH, N, D, L::BM, "dO")) != FA_OK) return rc;
   if ((rc = set_smem(fa::fa_bwd_sm100_kernel<D>, L::SMEM_ALLOC)) != FA_OK) return rc;
   fa::BwdParams p;
@@ -163,13 +164,14 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.B = B;
   p.H = H;
+  p.H_kv = H_kv;
   p.N = N;
   p.N_pad = ws.n_pad;
   p.n_ktiles = (N + 127) / 128;
   p.scale = scale;
   p.scale2 = scale * kLog2e;
   p.causal = causal ? 1 : 0;
-  const long long grid = static_cast<long long>(p.n_ktiles) * BH;
+  const long long grid = static_cast<long long>(p.n_ktiles) * B * H_kv;  // one CTA per K/V tile
   if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
   fa::fa_bwd_sm100_kernel<D><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
   return check_launch("fa_bwd_sm100_kernel");
@@ -193,15 +195,28 @@ int fa_device_status(unsigned int* code) {
   return FA_OK;
 }
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-           int N, int d, float scale, int causal, const uint8_t* block_mask,
-           const int32_t* kv_len, int dtype, void* stream) {
+}  // extern "C"
+
+namespace {
+
+int check_groups(int H, int H_kv) {
+  if (H_kv < 1 || H_kv > H || H % H_kv != 0)
+    return fail(FA_ERR_INVALID, "H = %d must be a positive multiple of H_kv = %d", H, H_kv);
+  return FA_OK;
+}
+
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int H_kv, int N, int d, float scale, int causal, const uint8_t* block_mask,
+             const int32_t* kv_len, int dtype, void* stream) {
   int rc = common_checks(q, k, v, o, lse, B, H, N, d, scale);
   if (rc != FA_OK) return rc;
+  if ((rc = check_groups(H, H_kv)) != FA_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == FA_BF16) {
-    if (d == 64) return launch_fwd<64>(q, k, v, o, lse, B, H, N, scale, causal, block_mask, kv_len, s);
-    if (d == 128) return launch_fwd<128>(q, k, v, o, lse, B, H, N, scale, causal, block_mask, kv_len, s);
+    if (d == 64)
+      return launch_fwd<64>(q, k, v, o, lse, B, H, H_kv, N, scale, causal, block_mask, kv_len, s);
+    if (d == 128)
+      return launch_fwd<128>(q, k, v, o, lse, B, H, H_kv, N, scale, causal, block_mask, kv_len, s);
     return fail(FA_ERR_UNSUPPORTED, "bf16 forward supports d in {64, 128}, got %d", d);
   }
   if (dtype == FA_F32) {
@@ -209,23 +224,20 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
     const long long rows = static_cast<long long>(B) * H * N;
     fa::fa_fwd_rowwarp_kernel<float, false><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
         static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-        static_cast<float*>(o), lse, block_mask, kv_len, B, H, N, d, scale, causal ? 1 : 0, 128, 0);
+        static_cast<float*>(o), lse, block_mask, kv_len, B, H, N, d, scale, causal ? 1 : 0, 128, 0,
+        H_kv);
     return check_launch("fa_fwd_rowwarp_kernel<f32>");
   }
   return fail(FA_ERR_INVALID, "unknown dtype %d", dtype);
 }
 
-size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
-  return bwd_ws(B, H, N, d).total;
-}
-
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-           const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
-           float scale, int causal, const uint8_t* block_mask, const int32_t* kv_len,
-           int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* dO, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
+             float scale, int causal, const uint8_t* block_mask, const int32_t* kv_len,
+             int dtype, void* workspace, size_t workspace_bytes, void* stream) {
   int rc = common_checks(q, k, v, o, lse, B, H, N, d, scale);
   if (rc != FA_OK) return rc;
+  if ((rc = check_groups(H, H_kv)) != FA_OK) return rc;
   if (!dO || !dq || !dk || !dv) return fail(FA_ERR_INVALID, "null gradient pointer");
   if (!aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return fail(FA_ERR_ALIGN, "gradient pointers must be 16-byte aligned");
@@ -249,14 +261,54 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
       reinterpret_cast<float*>(wsb + ws.dq), BH, N, ws.n_pad, d);
   if ((rc = check_launch("bwd_preprocess_kernel")) != FA_OK) return rc;
   if (d == 64)
-    rc = launch_bwd<64>(q, k, v, dO, dk, dv, B, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+    rc = launch_bwd<64>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
   else
-    rc = launch_bwd<128>(q, k, v, dO, dk, dv, B, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+    rc = launch_bwd<128>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
   if (rc != FA_OK) return rc;
   const long long n = static_cast<long long>(BH) * N * d;
   fa::dq_convert_kernel<<<static_cast<unsigned>((n / 8 + 255) / 256 + 1), 256, 0, s>>>(
       reinterpret_cast<const float*>(wsb + ws.dq), static_cast<__nv_bfloat16*>(dq), n, scale);
   return check_launch("dq_convert_kernel");
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+           int N, int d, float scale, int causal, const uint8_t* block_mask,
+           const int32_t* kv_len, int dtype, void* stream) {
+  return fwd_impl(q, k, v, o, lse, B, H, H, N, d, scale, causal, block_mask, kv_len, dtype,
+                  stream);
+}
+
+int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int H_kv, int N, int d, float scale, int causal, const uint8_t* block_mask,
+               const int32_t* kv_len, int dtype, void* stream) {
+  return fwd_impl(q, k, v, o, lse, B, H, H_kv, N, d, scale, causal, block_mask, kv_len, dtype,
+                  stream);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
+  return bwd_ws(B, H, N, d).total;
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+           float scale, int causal, const uint8_t* block_mask, const int32_t* kv_len,
+           int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, H, N, d, scale, causal, block_mask,
+                  kv_len, dtype, workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dO, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N,
+               int d, float scale, int causal, const uint8_t* block_mask,
+               const int32_t* kv_len, int dtype, void* workspace, size_t workspace_bytes,
+               void* stream) {
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, scale, causal, block_mask,
+                  kv_len, dtype, workspace, workspace_bytes, stream);
 }
 
 int fa_fwd_tile_reference(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -274,7 +326,7 @@ int fa_fwd_tile_reference(const void* q, const void* k, const void* v, void* o, 
       <<<static_cast<unsigned>((rows + 7) / 8), 256, 0, static_cast<cudaStream_t>(stream)>>>(
           static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
           static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), lse, block_mask,
-          kv_len, B, H, N, d, scale, causal ? 1 : 0, bc, flags);
+          kv_len, B, H, N, d, scale, causal ? 1 : 0, bc, flags, H);
   return check_launch("fa_fwd_rowwarp_kernel<bf16>");
 }
 
@@ -405,9 +457,9 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
       reinterpret_cast<float*>(wsb + ws.dq), BH, N, ws.n_pad, d);
   if ((rc = check_launch("bwd_preprocess_kernel")) != FA_OK) return rc;
   if (d == 64)
-    rc = launch_bwd<64>(q, k, v, dO, dk, dv, B, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+    rc = launch_bwd<64>(q, k, v, dO, dk, dv, B, H, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
   else
-    rc = launch_bwd<128>(q, k, v, dO, dk, dv, B, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+    rc = launch_bwd<128>(q, k, v, dO, dk, dv, B, H, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
   if (rc != FA_OK) return rc;
   const long long n = static_cast<long long>(BH) * N * d;
   fa::dq_convert_kernel<<<static_cast<unsigned>((n / 8 + 255) / 256 + 1), 256, 0, s>>>(

@@ -43,6 +43,7 @@ struct BwdParams {
   __nv_bfloat16* dk;          // [B*H][N][D]
   __nv_bfloat16* dv;          // [B*H][N][D]
   int B, H, N, N_pad;
+  int H_kv;                   // K/V heads: query heads G*j .. G*j+G-1 (G = H / H_kv) read head j
   int n_ktiles;               // ceil(N / 128)
   float scale, scale2;
   int causal;
@@ -125,10 +126,12 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int BH = p.B * p.H;
-  const int jt = static_cast<int>(blockIdx.x) / BH;  // KV tile; small jt (most work) first
-  const int bh = static_cast<int>(blockIdx.x) % BH;
-  const int b = bh / p.H;
+  const int G = p.H / p.H_kv;                         // query heads per K/V head
+  const int BHkv = p.B * p.H_kv;
+  const int jt = static_cast<int>(blockIdx.x) / BHkv;  // KV tile; small jt (most work) first
+  const int bhk = static_cast<int>(blockIdx.x) % BHkv;  // (b, K/V head)
+  const int b = bhk / p.H_kv;
+  const int bhq0 = b * p.H + (bhk % p.H_kv) * G;       // first query head of the group
   const int N = p.N;
   const int k0 = jt * 128;
   int kvlen = N;
@@ -146,12 +149,16 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       return false;
     return true;
   };
-  // steps of this CTA: a closed form unless a block mask decides tile by tile (a loop over all
-  // query tiles in every thread costs thousands of cycles per CTA at N = 16384)
+  // The CTA walks the query tiles it_first .. n_qt-1 of each of the G query heads of its group
+  // (work item w: head g = w / span, tile it_first + w % span); dK and dV of the shared K/V
+  // head accumulate over all of them.  Steps: a closed form unless a block mask decides tile by
+  // tile (a loop over all query tiles in every thread costs thousands of cycles at N = 16384).
   const int it_first = p.causal ? k0 / BM : 0;  // query tiles before it_first see no key here
+  const int span = n_qt - it_first;
   int n_steps = 0;
-  if (p.block_mask == nullptr) n_steps = kv_live ? n_qt - it_first : 0;
+  if (p.block_mask == nullptr) n_steps = kv_live ? span : 0;
   else for (int it = it_first; it < n_qt; ++it) n_steps += q_active(it) ? 1 : 0;
+  n_steps *= G;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv, 1);
@@ -190,12 +197,15 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       tma_prefetch_desc(&tm_do);
       mbar_arrive_expect_tx(bar_kv, 2 * L::KV_TILE);
       for (int s = 0; s < L::SUB; ++s) {
-        tma_load_3d(smem + L::OFF_K + s * L::KV_SUBTILE, &tm_k, bar_kv, s * 64, k0, bh);
-        tma_load_3d(smem + L::OFF_V + s * L::KV_SUBTILE, &tm_v, bar_kv, s * 64, k0, bh);
+        tma_load_3d(smem + L::OFF_K + s * L::KV_SUBTILE, &tm_k, bar_kv, s * 64, k0, bhk);
+        tma_load_3d(smem + L::OFF_V + s * L::KV_SUBTILE, &tm_v, bar_kv, s * 64, k0, bhk);
       }
       int t = 0;
-      for (int it = it_first; it < n_qt; ++it) {
+      for (int w = 0; w < G * span; ++w) {
+        const int g = w / span;
+        const int it = it_first + (w - g * span);
         if (!q_active(it)) continue;
+        const int bh = bhq0 + g;              // query head of this step
         const int st = t % L::QST;
         if (t >= L::QST &&
             !mbar_wait(&bar_qe[st], ((t / L::QST) - 1) & 1, abort_flag, SITE_BWD_LOAD_EMPTY))
@@ -352,7 +362,9 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     const float scale2 = p.scale2;
     bool ok = true;
     int t = 0;
-    for (int it = it_first; it < n_qt; ++it) {
+    for (int w = 0; w < G * span; ++w) {
+      const int g = w / span;
+      const int it = it_first + (w - g * span);
       if (!q_active(it)) continue;
       const int st = t % L::QST;
       const int buf = t & 1;
@@ -483,7 +495,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (ok) {
       const uint32_t col0 = h == 0 ? L::DV_COL : L::DK_COL;
       const float mul = h == 0 ? 1.0f : p.scale;
-      __nv_bfloat16* dst_row = (h == 0 ? p.dv : p.dk) + (static_cast<size_t>(bh) * N + kj) * D;
+      __nv_bfloat16* dst_row = (h == 0 ? p.dv : p.dk) + (static_cast<size_t>(bhk) * N + kj) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t g[32];
@@ -512,8 +524,11 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int qw = warp & 3;
     const uint32_t t_lane = static_cast<uint32_t>(32 * qw) << 16;
     int t = 0;
-    for (int it = it_first; it < n_qt; ++it) {
+    for (int w = 0; w < G * span; ++w) {
+      const int g = w / span;
+      const int it = it_first + (w - g * span);
       if (!q_active(it)) continue;
+      const int bh = bhq0 + g;                // query head of this step
       const int buf = t & 1;
       const int i0 = it * BM;
       const bool got = mbar_wait(&bar_dqf[buf], (t >> 1) & 1, abort_flag, SITE_BWD_DQ);

@@ -43,6 +43,7 @@ struct FwdParams {
   __nv_bfloat16* o;           // [B*H][N][D]
   float* lse;                 // [B*H][N]
   int B, H, N;
+  int H_kv;                   // K/V heads; query head h reads K/V head h / (H / H_kv)
   int n_mtiles;               // ceil(N / 256)
   float scale2;               // scale * log2(e)
   int causal;
@@ -108,6 +109,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int mt = p.n_mtiles - 1 - static_cast<int>(blockIdx.x) / BH;  // heaviest tiles first
   const int bh = static_cast<int>(blockIdx.x) % BH;
   const int b = bh / p.H;
+  const int bh_kv = b * p.H_kv + (bh % p.H) / (p.H / p.H_kv);  // K/V head of this query head
   const int N = p.N;
   const int m0 = mt * 256;
   int kvlen = N;
@@ -183,7 +185,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_arrive_expect_tx(&bar_kf[ks], L::TILE);
         for (int s = 0; s < L::SUB; ++s)
           tma_load_3d(smem + L::OFF_K + ks * L::TILE + s * L::SUBTILE, &tm_k, &bar_kf[ks], s * 64,
-                      j * 128, bh);
+                      j * 128, bh_kv);
         ++kn;
         if (vn >= L::VST &&
             !mbar_wait(&bar_ve[vs], ((vn / L::VST) - 1) & 1, abort_flag, SITE_FWD_LOAD_EMPTY))
@@ -191,7 +193,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_arrive_expect_tx(&bar_vf[vs], L::TILE);
         for (int s = 0; s < L::SUB; ++s)
           tma_load_3d(smem + L::OFF_V + vs * L::TILE + s * L::SUBTILE, &tm_v, &bar_vf[vs], s * 64,
-                      j * 128, bh);
+                      j * 128, bh_kv);
         ++vn;
       }
       // Never leave the CTA with a copy in flight: wait for the last loads of every stage

@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(256)
 fa_fwd_rowwarp_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                       T* __restrict__ o, float* __restrict__ lse, const uint8_t* block_mask,
                       const int32_t* kv_len, int B, int H, int N, int d, float scale, int causal,
-                      int bc, int flags) {
+                      int bc, int flags, int H_kv) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row_g = static_cast<long long>(blockIdx.x) * 8 + warp;  // flat bh*N + i
   if (row_g >= static_cast<long long>(B) * H * N) return;
@@ -63,8 +63,9 @@ fa_fwd_rowwarp_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
   if (kv_len != nullptr) kvlen = min(max(kv_len[b], 0), N);
   const int nb = (N + 127) / 128;
   const T* qi = q + row_g * d;
-  const T* kh = k + static_cast<size_t>(bh) * N * d;
-  const T* vh = v + static_cast<size_t>(bh) * N * d;
+  const int bh_kv = b * H_kv + (bh % H) / (H / H_kv);  // K/V head of query head bh
+  const T* kh = k + static_cast<size_t>(bh_kv) * N * d;
+  const T* vh = v + static_cast<size_t>(bh_kv) * N * d;
   const int ncol = (d + 31) / 32;  // <= 4
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   float m = -INFINITY, l = 0.f;

@@ -108,6 +108,26 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                    float scale, int causal, const uint8_t* block_mask, const int32_t* kv_len,
                    int dtype, void* stream);
 
+/*
+ * Grouped-query and multi-query attention (the MQA/GQA of the tcdigital FA-2 ROI article, section
+ * "MQA/GQA ... との相乗効果"): H query heads share H_kv K/V heads, H a multiple of H_kv, and query
+ * head h reads K/V head h / (H / H_kv) (contiguous groups; H_kv = 1 is multi-query attention).
+ * q, o, dO, dq are [B][H][N][d]; k, v, dk, dv are [B][H_kv][N][d]; lse is [B][H][N].
+ * Everything else -- dtypes, masks, alignment, status codes -- is as for fa_fwd / fa_bwd; the
+ * workspace of fa_bwd_gqa is fa_bwd_workspace_size(B, H, N, d) (query heads).  fa_bwd_gqa
+ * accumulates dK and dV of a shared head over its query heads on chip, in a fixed order, so
+ * they stay deterministic.  H_kv < 1, H_kv > H or H % H_kv != 0 give FA_ERR_INVALID.
+ * fa_fwd_gqa with H_kv = H is fa_fwd; fa_bwd_gqa with H_kv = H is fa_bwd.
+ */
+int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int H_kv, int N, int d, float scale, int causal, const uint8_t* block_mask,
+               const int32_t* kv_len, int dtype, void* stream);
+int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dO, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N,
+               int d, float scale, int causal, const uint8_t* block_mask,
+               const int32_t* kv_len, int dtype, void* workspace, size_t workspace_bytes,
+               void* stream);
+
 /* Flags of fa_fwd_tile_reference: the other two axes of the deviation study. */
 enum {
   FA_TILE_REVERSE = 1,    /* visit the key tiles from the last to the first */

@@ -93,6 +93,20 @@ def test_bwd_validation_codes(lib):
     assert "256-byte" in lib.fa_get_last_error().decode()
 
 
+def test_gqa_validation_codes(lib):
+    def fwd(H=4, H_kv=2):
+        return lib.fa_fwd_gqa(A, A, A, A, A, 1, H, H_kv, 128, 64, 0.125, 1, None, None, 0, None)
+
+    def bwd(H=4, H_kv=2, wsb=1 << 30):
+        return lib.fa_bwd_gqa(A, A, A, A, A, A, A, A, A, 1, H, H_kv, 256, 64, 0.125, 1, None,
+                              None, 0, A, wsb, None)
+    for H, H_kv in ((4, 3), (4, 0), (4, 8), (6, -2)):
+        assert fwd(H, H_kv) == INVALID
+        assert "H_kv" in lib.fa_get_last_error().decode()
+        assert bwd(H, H_kv) == INVALID
+    assert bwd(wsb=10) == WORKSPACE
+
+
 def test_aux_entry_validation(lib):
     assert lib.fa_fwd_tile_reference(A, A, A, A, A, 1, 1, 64, 64, 0.125, 0, None, None, 48, 0,
                                      None) == INVALID
