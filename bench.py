@@ -385,6 +385,33 @@ def deviation_sweep():
     return out
 
 
+def deterministic_measurement(x, g, o, lse, iters: int = 10):
+    """fa_bwd_deterministic on the bench workload: dQ from the query-stationary kernel, no
+    atomics.  Reported against the same algorithmic backward FLOPs (10 d per pair) as fa_bwd,
+    and against the FLOPs it executes (14 d per pair: S and dP are computed twice)."""
+    import exact_io_aware_98_b200 as fa
+    H = x["q"].shape[1]
+    B, N, d = x["B"], x["N"], x["d"]
+    _, f_bwd = flops(x, H)
+    ws = torch.empty(fa.bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=g["q"].device)
+    dq, dk, dv = (torch.empty_like(g["q"]) for _ in range(3))
+    kw = dict(scale=g["scale"], causal=g["causal"], block_mask=g["block_mask"],
+              kv_len=g["kv_len"], workspace=ws, dq=dq, dk=dk, dv=dv, deterministic=True)
+    for _ in range(3):
+        fa.bwd(g["q"], g["k"], g["v"], o, lse, g["do"], **kw)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        fa.bwd(g["q"], g["k"], g["v"], o, lse, g["do"], **kw)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / iters
+    return {"ms": round(ms, 4), "tflops_algorithmic": round(f_bwd / ms / 1e9, 2),
+            "tflops_executed": round(1.4 * f_bwd / ms / 1e9, 2),
+            "device_status": fa.device_status(),
+            "note": "dK/dV by the main kernel without dQ, dQ by fa_bwd_dq_sm100_kernel"}
+
+
 def gqa_measurement(iters: int = 10):
     """Grouped-query attention (the MQA/GQA of the tcdigital FA-2 ROI article) on a Llama-class
     grouping: B1 H32 H_kv8 N8192 d128 causal.  FLOPs count per query head, as for attention with
@@ -476,6 +503,7 @@ def main():
             line["cpu_baseline"] = cpu
             line["max_err_vs_fp64"] = err
             line["deviation_sweep"] = deviation_sweep()
+            line["bwd_deterministic"] = deterministic_measurement(x, g, o, lse)
             line["gqa"] = gqa_measurement()
         if rank == 0:
             print(json.dumps(line), flush=True)

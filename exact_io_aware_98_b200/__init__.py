@@ -29,6 +29,8 @@ SIGNATURES = {
     "fa_bwd_workspace_size": (_sz, [_i, _i, _i, _i]),
     "fa_bwd_gqa": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i,
                         _vp, _vp, _i, _vp, _sz, _vp]),
+    "fa_bwd_deterministic": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                                  _f, _i, _vp, _vp, _i, _vp, _sz, _vp]),
     "fa_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp,
                     _vp, _i, _vp, _sz, _vp]),
     "fa_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
@@ -154,9 +156,11 @@ def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
 
 
 def bwd(q, k, v, o, lse, do, scale: Optional[float] = None, causal: bool = False,
-        block_mask=None, kv_len=None, workspace=None, dq=None, dk=None, dv=None):
-    """dQ, dK, dV = fa_bwd(...); bf16 tensors on the GPU, q/o/do [B, H, N, d], k/v and dK/dV
-    [B, H_kv, N, d] (fa_bwd_gqa when H_kv < H)."""
+        block_mask=None, kv_len=None, workspace=None, dq=None, dk=None, dv=None,
+        deterministic: bool = False):
+    """dQ, dK, dV = fa_bwd(...); tensors on the GPU, q/o/do [B, H, N, d], k/v and dK/dV
+    [B, H_kv, N, d] (fa_bwd_gqa when H_kv < H).  ``deterministic`` calls fa_bwd_deterministic:
+    bit-reproducible gradients, dQ without atomics."""
     lib = load()
     B, H, N, d = q.shape
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
@@ -175,7 +179,13 @@ def bwd(q, k, v, o, lse, do, scale: Optional[float] = None, causal: bool = False
         raise FaError("gradient shapes must match q, k and v")
     bm, kl = _masks(block_mask, kv_len)
     s = default_scale(d) if scale is None else float(scale)
-    if H_kv == H:
+    if deterministic:
+        rc = lib.fa_bwd_deterministic(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do),
+                                      _ptr(dq), _ptr(dk), _ptr(dv), B, H, H_kv, N, d, s,
+                                      int(causal), bm, kl, _dtype_code(q), _ptr(ws), ws.numel(),
+                                      _stream())
+        _check(rc, "fa_bwd_deterministic")
+    elif H_kv == H:
         rc = lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq),
                         _ptr(dk), _ptr(dv), B, H, N, d, s, int(causal), bm, kl, _dtype_code(q),
                         _ptr(ws), ws.numel(), _stream())

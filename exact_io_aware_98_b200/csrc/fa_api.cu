@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_bwd_dq_sm100.cuh"
 #include "fa_bwd_sm100.cuh"
 #include "fa_fwd_sm100.cuh"
 #include "fa_simt.cuh"
@@ -141,7 +142,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   return check_launch("fa_fwd_sm100_kernel");
 }
 
-template <int D>
+template <int D, bool WITH_DQ>
 int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
                int B, int H, int H_kv, int N, float scale, int causal, const uint8_t* bm,
                const int32_t* kv_len, const BwdWs& ws, uint8_t* wsb, cudaStream_t stream) {
@@ -153,7 +154,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void
   if ((rc = make_map(&mk, k, B * H_kv, N, D, 128, "k")) != FA_OK) return rc;
   if ((rc = make_map(&mv, v, B * H_kv, N, D, 128, "v")) != FA_OK) return rc;
   if ((rc = make_map(&mdo, dO, BH, N, D, L::BM, "dO")) != FA_OK) return rc;
-  if ((rc = set_smem(fa::fa_bwd_sm100_kernel<D>, L::SMEM_ALLOC)) != FA_OK) return rc;
+  if ((rc = set_smem(fa::fa_bwd_sm100_kernel<D, WITH_DQ>, L::SMEM_ALLOC)) != FA_OK) return rc;
   fa::BwdParams p;
   p.block_mask = bm;
   p.kv_len = kv_len;
@@ -173,8 +174,43 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void
   p.causal = causal ? 1 : 0;
   const long long grid = static_cast<long long>(p.n_ktiles) * B * H_kv;  // one CTA per K/V tile
   if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
-  fa::fa_bwd_sm100_kernel<D><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
+  fa::fa_bwd_sm100_kernel<D, WITH_DQ><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
   return check_launch("fa_bwd_sm100_kernel");
+}
+
+// dQ without atomics: one CTA per 128 query rows walks the KV tiles (fa_bwd_dq_sm100.cuh).
+template <int D>
+int launch_bwd_dq(const void* q, const void* k, const void* v, const void* dO, void* dq, int B,
+                  int H, int H_kv, int N, float scale, int causal, const uint8_t* bm,
+                  const int32_t* kv_len, const BwdWs& ws, uint8_t* wsb, cudaStream_t stream) {
+  using L = fa::BwdDqLayout<D>;
+  CUtensorMap mq, mk, mv, mdo;
+  const int BH = B * H;
+  int rc;
+  if ((rc = make_map(&mq, q, BH, N, D, 128, "q")) != FA_OK) return rc;
+  if ((rc = make_map(&mk, k, B * H_kv, N, D, 128, "k")) != FA_OK) return rc;
+  if ((rc = make_map(&mv, v, B * H_kv, N, D, 128, "v")) != FA_OK) return rc;
+  if ((rc = make_map(&mdo, dO, BH, N, D, 128, "dO")) != FA_OK) return rc;
+  if ((rc = set_smem(fa::fa_bwd_dq_sm100_kernel<D>, L::SMEM_ALLOC)) != FA_OK) return rc;
+  fa::BwdDqParams p;
+  p.block_mask = bm;
+  p.kv_len = kv_len;
+  p.lse2 = reinterpret_cast<const float*>(wsb + ws.lse2);
+  p.dvec = reinterpret_cast<const float*>(wsb + ws.dvec);
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.B = B;
+  p.H = H;
+  p.H_kv = H_kv;
+  p.N = N;
+  p.N_pad = ws.n_pad;
+  p.n_mtiles = (N + 127) / 128;
+  p.scale = scale;
+  p.scale2 = scale * kLog2e;
+  p.causal = causal ? 1 : 0;
+  const long long grid = static_cast<long long>(p.n_mtiles) * BH;
+  if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
+  fa::fa_bwd_dq_sm100_kernel<D><<<static_cast<unsigned>(grid), 320, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
+  return check_launch("fa_bwd_dq_sm100_kernel");
 }
 
 }  // namespace
@@ -234,18 +270,19 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
 int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse,
              const void* dO, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
              float scale, int causal, const uint8_t* block_mask, const int32_t* kv_len,
-             int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+             int dtype, void* workspace, size_t workspace_bytes, void* stream,
+             bool deterministic) {
   int rc = common_checks(q, k, v, o, lse, B, H, N, d, scale);
   if (rc != FA_OK) return rc;
   if ((rc = check_groups(H, H_kv)) != FA_OK) return rc;
   if (!dO || !dq || !dk || !dv) return fail(FA_ERR_INVALID, "null gradient pointer");
   if (!aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return fail(FA_ERR_ALIGN, "gradient pointers must be 16-byte aligned");
-  if (dtype != FA_BF16) {
-    if (dtype == FA_F32) return fail(FA_ERR_UNSUPPORTED, "fp32 backward is not built");
-    return fail(FA_ERR_INVALID, "unknown dtype %d", dtype);
-  }
-  if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "bf16 backward supports d in {64, 128}, got %d", d);
+  if (dtype != FA_BF16 && dtype != FA_F32) return fail(FA_ERR_INVALID, "unknown dtype %d", dtype);
+  if (dtype == FA_F32 && d > 128)
+    return fail(FA_ERR_UNSUPPORTED, "fp32 backward supports d <= 128, got %d", d);
+  if (dtype == FA_BF16 && d != 64 && d != 128)
+    return fail(FA_ERR_UNSUPPORTED, "bf16 backward supports d in {64, 128}, got %d", d);
   const BwdWs ws = bwd_ws(B, H, N, d);
   if (workspace == nullptr || workspace_bytes < ws.total)
     return fail(FA_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", ws.total, workspace_bytes);
@@ -254,16 +291,46 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   const int BH = B * H;
+  if (dtype == FA_F32) {
+    // CUDA-core fp32 backward: Dvec, then dQ per query row and dK/dV per key row (no atomics)
+    const long long qrows = static_cast<long long>(BH) * N;
+    const long long krows = static_cast<long long>(B) * H_kv * N;
+    float* dvec = reinterpret_cast<float*>(wsb + ws.dvec);
+    fa::bwd_dvec_f32_kernel<<<static_cast<unsigned>((qrows + 7) / 8), 256, 0, s>>>(
+        static_cast<const float*>(o), static_cast<const float*>(dO), dvec, qrows, d);
+    if ((rc = check_launch("bwd_dvec_f32_kernel")) != FA_OK) return rc;
+    fa::fa_bwd_f32_dq_kernel<<<static_cast<unsigned>((qrows + 7) / 8), 256, 0, s>>>(
+        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+        static_cast<const float*>(dO), lse, dvec, static_cast<float*>(dq), block_mask, kv_len, B,
+        H, H_kv, N, d, scale, causal ? 1 : 0);
+    if ((rc = check_launch("fa_bwd_f32_dq_kernel")) != FA_OK) return rc;
+    fa::fa_bwd_f32_dkdv_kernel<<<static_cast<unsigned>((krows + 7) / 8), 256, 0, s>>>(
+        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+        static_cast<const float*>(dO), lse, dvec, static_cast<float*>(dk), static_cast<float*>(dv),
+        block_mask, kv_len, B, H, H_kv, N, d, scale, causal ? 1 : 0);
+    return check_launch("fa_bwd_f32_dkdv_kernel");
+  }
   const long long pre_rows = static_cast<long long>(BH) * ws.n_pad;
   fa::bwd_preprocess_kernel<<<static_cast<unsigned>((pre_rows + 7) / 8), 256, 0, s>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse,
       reinterpret_cast<float*>(wsb + ws.lse2), reinterpret_cast<float*>(wsb + ws.dvec),
-      reinterpret_cast<float*>(wsb + ws.dq), BH, N, ws.n_pad, d);
+      deterministic ? nullptr : reinterpret_cast<float*>(wsb + ws.dq), BH, N, ws.n_pad, d);
   if ((rc = check_launch("bwd_preprocess_kernel")) != FA_OK) return rc;
+  if (deterministic) {
+    // dK and dV by the main kernel without its dQ part, dQ by the query-stationary kernel
+    if (d == 64)
+      rc = launch_bwd<64, false>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+    else
+      rc = launch_bwd<128, false>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+    if (rc != FA_OK) return rc;
+    if (d == 64)
+      return launch_bwd_dq<64>(q, k, v, dO, dq, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+    return launch_bwd_dq<128>(q, k, v, dO, dq, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+  }
   if (d == 64)
-    rc = launch_bwd<64>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+    rc = launch_bwd<64, true>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
   else
-    rc = launch_bwd<128>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+    rc = launch_bwd<128, true>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
   if (rc != FA_OK) return rc;
   const long long n = static_cast<long long>(BH) * N * d;
   fa::dq_convert_kernel<<<static_cast<unsigned>((n / 8 + 255) / 256 + 1), 256, 0, s>>>(
@@ -299,7 +366,7 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            float scale, int causal, const uint8_t* block_mask, const int32_t* kv_len,
            int dtype, void* workspace, size_t workspace_bytes, void* stream) {
   return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, H, N, d, scale, causal, block_mask,
-                  kv_len, dtype, workspace, workspace_bytes, stream);
+                  kv_len, dtype, workspace, workspace_bytes, stream, false);
 }
 
 int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -308,7 +375,16 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const
                const int32_t* kv_len, int dtype, void* workspace, size_t workspace_bytes,
                void* stream) {
   return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, scale, causal, block_mask,
-                  kv_len, dtype, workspace, workspace_bytes, stream);
+                  kv_len, dtype, workspace, workspace_bytes, stream, false);
+}
+
+int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
+                         int H, int H_kv, int N, int d, float scale, int causal,
+                         const uint8_t* block_mask, const int32_t* kv_len, int dtype,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, scale, causal, block_mask,
+                  kv_len, dtype, workspace, workspace_bytes, stream, true);
 }
 
 int fa_fwd_tile_reference(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -457,9 +533,9 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
       reinterpret_cast<float*>(wsb + ws.dq), BH, N, ws.n_pad, d);
   if ((rc = check_launch("bwd_preprocess_kernel")) != FA_OK) return rc;
   if (d == 64)
-    rc = launch_bwd<64>(q, k, v, dO, dk, dv, B, H, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+    rc = launch_bwd<64, true>(q, k, v, dO, dk, dv, B, H, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
   else
-    rc = launch_bwd<128>(q, k, v, dO, dk, dv, B, H, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+    rc = launch_bwd<128, true>(q, k, v, dO, dk, dv, B, H, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
   if (rc != FA_OK) return rc;
   const long long n = static_cast<long long>(BH) * N * d;
   fa::dq_convert_kernel<<<static_cast<unsigned>((n / 8 + 255) / 256 + 1), 256, 0, s>>>(

@@ -226,7 +226,8 @@ naive_pv_kernel(const __nv_bfloat16* __restrict__ pm, const __nv_bfloat16* __res
 
 // ---------------------------------------------------------------------------- backward helpers
 // Dvec_i = sum_c dO_ic O_ic (fp32); lse2_i = lse_i * log2(e) (+inf for rows with no key and for
-// the padding rows N..N_pad-1); zeroes the fp32 dQ accumulator.  One warp per row of N_pad.
+// the padding rows N..N_pad-1); zeroes the fp32 dQ accumulator unless dq_acc is null (the
+// deterministic backward has none).  One warp per row of N_pad.
 __global__ void __launch_bounds__(256)
 bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
                       const float* __restrict__ lse, float* __restrict__ lse2,
@@ -247,7 +248,8 @@ bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* 
   float acc = 0.f;
   for (int c = lane; c < d; c += 32) acc = fmaf(__bfloat162float(dO[off + c]), __bfloat162float(o[off + c]), acc);
   for (int offs = 16; offs > 0; offs >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, offs);
-  for (int c = lane; c < d; c += 32) dq_acc[off + c] = 0.f;
+  if (dq_acc != nullptr)
+    for (int c = lane; c < d; c += 32) dq_acc[off + c] = 0.f;
   if (lane == 0) {
     const float ls = lse[static_cast<size_t>(bh) * N + i];
     lse2[r] = (ls == -INFINITY) ? INFINITY : ls * 1.4426950408889634f;
@@ -275,6 +277,163 @@ dq_convert_kernel(const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ 
     *reinterpret_cast<uint4*>(dq + e) = u;
   } else {
     for (long long x = e; x < n; ++x) dq[x] = __float2bfloat16_rn(dq_acc[x] * scale);
+  }
+}
+
+// ---------------------------------------------------------------------------- fp32 backward
+// The backward of the fp32 path on CUDA cores, with the recompute form of the tensor-core
+// backward: P_ij = exp(s_ij - lse_i), dS_ij = P_ij (dO_i . v_j - Dvec_i), Dvec_i = dO_i . O_i.
+// Two kernels, each owning its output rows, so every sum runs in a fixed order (no atomics):
+// the gradients are deterministic.  Query head h reads K/V head h / (H / H_kv).
+
+// Dvec_i = sum_c dO_ic O_ic in fp32.  One warp per query row.
+__global__ void __launch_bounds__(256)
+bwd_dvec_f32_kernel(const float* __restrict__ o, const float* __restrict__ dO,
+                    float* __restrict__ dvec, long long rows, int d) {
+  const long long r = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  float acc = 0.f;
+  for (int c = lane; c < d; c += 32) acc = fmaf(dO[r * d + c], o[r * d + c], acc);
+  for (int offs = 16; offs > 0; offs >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, offs);
+  if (lane == 0) dvec[r] = acc;
+}
+
+__device__ __forceinline__ float dot_f32(const float* __restrict__ a, const float* __restrict__ b,
+                                         int d) {
+  float s = 0.f;
+  for (int c = 0; c < d; ++c) s = fmaf(a[c], b[c], s);
+  return s;
+}
+
+// dQ_i = scale sum_j dS_ij k_j.  One warp per query row; lane l takes keys t0 + 32u + l of each
+// 256-key tile, then the warp accumulates output column 32cc + lane over the tile's keys.
+__global__ void __launch_bounds__(256)
+fa_bwd_f32_dq_kernel(const float* __restrict__ q, const float* __restrict__ k,
+                     const float* __restrict__ v, const float* __restrict__ dO,
+                     const float* __restrict__ lse, const float* __restrict__ dvec,
+                     float* __restrict__ dq, const uint8_t* block_mask, const int32_t* kv_len,
+                     int B, int H, int H_kv, int N, int d, float scale, int causal) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row_g = static_cast<long long>(blockIdx.x) * 8 + warp;  // flat bh*N + i
+  if (row_g >= static_cast<long long>(B) * H * N) return;
+  const int i = static_cast<int>(row_g % N);
+  const int bh = static_cast<int>(row_g / N);
+  const int b = bh / H;
+  const int bh_kv = b * H_kv + (bh % H) / (H / H_kv);
+  int kvlen = N;
+  if (kv_len != nullptr) kvlen = min(max(kv_len[b], 0), N);
+  const int nb = (N + 127) / 128;
+  const float* qi = q + row_g * d;
+  const float* doi = dO + row_g * d;
+  const float* kh = k + static_cast<size_t>(bh_kv) * N * d;
+  const float* vh = v + static_cast<size_t>(bh_kv) * N * d;
+  const float lse_i = lse[row_g];
+  const float dv_i = dvec[row_g];
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (lse_i != -INFINITY) {  // a row with no key has P = 0 everywhere
+    for (int t0 = 0; t0 < N; t0 += 256) {
+      float ds[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        ds[u] = 0.f;
+        const int j = t0 + 32 * u + lane;
+        if (j < N && key_allowed(i, j, kvlen, causal, block_mask, nb)) {
+          const float p = expf(dot_f32(qi, kh + static_cast<size_t>(j) * d, d) * scale - lse_i);
+          ds[u] = p * (dot_f32(doi, vh + static_cast<size_t>(j) * d, d) - dv_i);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        for (int src = 0; src < 32; ++src) {
+          const float w = __shfl_sync(0xffffffffu, ds[u], src);
+          const int j = t0 + 32 * u + src;
+          if (w == 0.f || j >= N) continue;
+          const float* kj = kh + static_cast<size_t>(j) * d;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            const int c = 32 * cc + lane;
+            if (c < d) acc[cc] = fmaf(w, kj[c], acc[cc]);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    const int c = 32 * cc + lane;
+    if (c < d) dq[row_g * d + c] = acc[cc] * scale;
+  }
+}
+
+// dV_j = sum_i P_ij dO_i and dK_j = scale sum_i dS_ij q_i over every query head of the K/V
+// head's group.  One warp per key row; lane l takes queries t0 + 32u + l of each 256-row tile.
+__global__ void __launch_bounds__(256)
+fa_bwd_f32_dkdv_kernel(const float* __restrict__ q, const float* __restrict__ k,
+                       const float* __restrict__ v, const float* __restrict__ dO,
+                       const float* __restrict__ lse, const float* __restrict__ dvec,
+                       float* __restrict__ dk, float* __restrict__ dv, const uint8_t* block_mask,
+                       const int32_t* kv_len, int B, int H, int H_kv, int N, int d, float scale,
+                       int causal) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row_g = static_cast<long long>(blockIdx.x) * 8 + warp;  // flat bh_kv*N + j
+  if (row_g >= static_cast<long long>(B) * H_kv * N) return;
+  const int j = static_cast<int>(row_g % N);
+  const int bh_kv = static_cast<int>(row_g / N);
+  const int b = bh_kv / H_kv;
+  const int G = H / H_kv;
+  int kvlen = N;
+  if (kv_len != nullptr) kvlen = min(max(kv_len[b], 0), N);
+  const int nb = (N + 127) / 128;
+  const float* kj = k + row_g * d;
+  const float* vj = v + row_g * d;
+  float acc_k[4] = {0.f, 0.f, 0.f, 0.f}, acc_v[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int g = 0; g < G && j < kvlen; ++g) {
+    const int bh = b * H + (bh_kv % H_kv) * G + g;  // query head of the group
+    const float* qh = q + static_cast<size_t>(bh) * N * d;
+    const float* doh = dO + static_cast<size_t>(bh) * N * d;
+    for (int t0 = 0; t0 < N; t0 += 256) {
+      float pv[8], ds[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        pv[u] = 0.f;
+        ds[u] = 0.f;
+        const int i = t0 + 32 * u + lane;
+        if (i < N && key_allowed(i, j, kvlen, causal, block_mask, nb)) {
+          const size_t r = static_cast<size_t>(bh) * N + i;
+          const float p = expf(dot_f32(qh + static_cast<size_t>(i) * d, kj, d) * scale - lse[r]);
+          pv[u] = p;
+          ds[u] = p * (dot_f32(doh + static_cast<size_t>(i) * d, vj, d) - dvec[r]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        for (int src = 0; src < 32; ++src) {
+          const float wp = __shfl_sync(0xffffffffu, pv[u], src);
+          const float ws = __shfl_sync(0xffffffffu, ds[u], src);
+          const int i = t0 + 32 * u + src;
+          if ((wp == 0.f && ws == 0.f) || i >= N) continue;
+          const float* qi = qh + static_cast<size_t>(i) * d;
+          const float* doi = doh + static_cast<size_t>(i) * d;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            const int c = 32 * cc + lane;
+            if (c < d) {
+              acc_v[cc] = fmaf(wp, doi[c], acc_v[cc]);
+              acc_k[cc] = fmaf(ws, qi[c], acc_k[cc]);
+            }
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    const int c = 32 * cc + lane;
+    if (c < d) {
+      dk[row_g * d + c] = acc_k[cc] * scale;
+      dv[row_g * d + c] = acc_v[cc];
+    }
   }
 }
 

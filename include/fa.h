@@ -74,11 +74,15 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 /*
  * fa_bwd -- backward pass of fa_fwd from (q, k, v, o, lse, dO), recomputing the scores:
  *   dV = A^T dO,  dS = A o (dO V^T - rowsum(dO o O)),  dQ = scale dS K,  dK = scale dS^T Q.
- *   Only FA_BF16 with d in {64, 128}.  o and lse must be fa_fwd's outputs for the same
- *   arguments.  workspace: device memory of at least fa_bwd_workspace_size() bytes, 256-byte
- *   aligned, owned by the caller, scratch only (its contents on entry do not matter).
- *   dq accumulates across key tiles with fp32 atomics, so its last bits may differ between
- *   runs; dk and dv are deterministic.
+ *   dtype FA_BF16: d in {64, 128}; tensor-core kernel.  dq accumulates across key tiles with
+ *                  fp32 atomics, so its last bits may differ between runs; dk and dv are
+ *                  deterministic.
+ *   dtype FA_F32 : 1 <= d <= 128; CUDA-core fp32 kernels (one warp per query row for dq, one
+ *                  per key row for dk and dv), exact expf, every sum in a fixed order: all
+ *                  three gradients are deterministic.
+ *   o and lse must be fa_fwd's outputs for the same arguments.  workspace: device memory of at
+ *   least fa_bwd_workspace_size() bytes, 256-byte aligned, owned by the caller, scratch only
+ *   (its contents on entry do not matter).
  */
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
            const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
@@ -127,6 +131,23 @@ int fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const
                int d, float scale, int causal, const uint8_t* block_mask,
                const int32_t* kv_len, int dtype, void* workspace, size_t workspace_bytes,
                void* stream);
+
+/*
+ * fa_bwd_deterministic -- fa_bwd_gqa with bit-reproducible gradients: the same inputs give the
+ * same dq, dk and dv bits on every run.  Arguments, layouts, workspace and errors are those of
+ * fa_bwd_gqa (H_kv = H for ordinary attention).
+ *   dtype FA_BF16: dk and dv come from the tensor-core backward without its dq part; dq comes
+ *                  from a second tensor-core kernel that owns 128 query rows per CTA and walks
+ *                  their KV tiles in increasing order, accumulating on chip -- no atomics.  It
+ *                  recomputes S and dP, so the call does 14 d FLOP per unmasked (row, key) pair
+ *                  instead of fa_bwd's 10 d.
+ *   dtype FA_F32 : the fp32 backward of fa_bwd, which is deterministic already.
+ */
+int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
+                         int H, int H_kv, int N, int d, float scale, int causal,
+                         const uint8_t* block_mask, const int32_t* kv_len, int dtype,
+                         void* workspace, size_t workspace_bytes, void* stream);
 
 /* Flags of fa_fwd_tile_reference: the other two axes of the deviation study. */
 enum {

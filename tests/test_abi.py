@@ -84,7 +84,7 @@ def test_bwd_validation_codes(lib):
                           ws if wsaddr is None else wsaddr, wsb, None)
     assert bwd(dq=None) == INVALID
     assert bwd(dq=A + 2) == ALIGN
-    assert bwd(dtype=1) == UNSUPPORTED
+    assert bwd(dtype=1, d=256) == UNSUPPORTED
     assert bwd(dtype=3) == INVALID
     assert bwd(d=32) == UNSUPPORTED
     assert bwd(ws=None) == WORKSPACE
@@ -105,6 +105,15 @@ def test_gqa_validation_codes(lib):
         assert "H_kv" in lib.fa_get_last_error().decode()
         assert bwd(H, H_kv) == INVALID
     assert bwd(wsb=10) == WORKSPACE
+
+    def det(H=4, H_kv=2, wsb=1 << 30, dtype=0, d=64):
+        return lib.fa_bwd_deterministic(A, A, A, A, A, A, A, A, A, 1, H, H_kv, 256, d, 0.125, 1,
+                                        None, None, dtype, A, wsb, None)
+    assert det(H_kv=3) == INVALID
+    assert det(wsb=10) == WORKSPACE
+    assert det(d=96) == UNSUPPORTED
+    assert det(dtype=1, d=256) == UNSUPPORTED
+    assert det(dtype=5) == INVALID
 
 
 def test_aux_entry_validation(lib):
