@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(syn.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="time fa_bwd_deterministic (dQ without atomics) as the step's backward")
     ap.add_argument("--cpu-rows", type=int, default=16384,
                     help="query rows in the oracle's timed sample")
     ap.add_argument("--ref-rows", type=int, default=1024,
@@ -200,9 +202,12 @@ def run_ours(args, rank: int, world: int, dist):
     kw = dict(scale=g["scale"], causal=g["causal"], block_mask=g["block_mask"],
               kv_len=g["kv_len"])
 
+    det = bool(args.deterministic)
+
     def step():
         fa.fwd(g["q"], g["k"], g["v"], out=o, lse=lse, **kw)
-        fa.bwd(g["q"], g["k"], g["v"], o, lse, g["do"], workspace=ws, dq=dq, dk=dk, dv=dv, **kw)
+        fa.bwd(g["q"], g["k"], g["v"], o, lse, g["do"], workspace=ws, dq=dq, dk=dk, dv=dv,
+               deterministic=det, **kw)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -221,7 +226,8 @@ def run_ours(args, rank: int, world: int, dist):
         ev[s][0].record()
         fa.fwd(g["q"], g["k"], g["v"], out=o, lse=lse, **kw)
         ev[s][1].record()
-        fa.bwd(g["q"], g["k"], g["v"], o, lse, g["do"], workspace=ws, dq=dq, dk=dk, dv=dv, **kw)
+        fa.bwd(g["q"], g["k"], g["v"], o, lse, g["do"], workspace=ws, dq=dq, dk=dk, dv=dv,
+               deterministic=det, **kw)
         ev[s][2].record()
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -251,7 +257,7 @@ def run_ours(args, rank: int, world: int, dist):
                 din[k].copy_(hin[k], non_blocking=True)
             fa.fwd(din["q"], din["k"], din["v"], out=o, lse=lse, **kw)
             fa.bwd(din["q"], din["k"], din["v"], o, lse, din["do"], workspace=ws, dq=dq, dk=dk,
-                   dv=dv, **kw)
+                   dv=dv, deterministic=det, **kw)
             for k, src in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
                 hout[k].copy_(src, non_blocking=True)
 
@@ -298,7 +304,8 @@ def run_ours(args, rank: int, world: int, dist):
         "config": {"workload": f"{args.workload}: {syn.WORKLOADS[args.workload].description}",
                    "B": B, "H": H, "N": N, "d": d,
                    "mask": syn.WORKLOADS[args.workload].mask,
-                   "step": "fa_fwd + fa_bwd", "parallelism": f"replicas x{world}",
+                   "step": "fa_fwd + " + ("fa_bwd_deterministic" if det else "fa_bwd"),
+                   "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2: Q,K,V,dO are 4 x %.0f MiB per step"
                          % (x["q"].numel() * 2 / 2**20)},
         "fwd": {"ms": round(fwd_ms, 4), "tflops": round(fwd_tf, 2),
@@ -307,6 +314,7 @@ def run_ours(args, rank: int, world: int, dist):
                 "frac_sustained": round(bwd_tf / sustained, 4)},
         "roofline": roof,
         "clocks": clocks,
+        # per step: fa_fwd's kernel + preprocess, main backward and dQ convert (or dQ kernel)
         "gpu_launches": K * 4,
         "device_status": status,
         "e2e": e2e,

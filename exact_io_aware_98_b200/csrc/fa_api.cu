@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_bwd_dkdv_sm100.cuh"
 #include "fa_bwd_dq_sm100.cuh"
 #include "fa_bwd_sm100.cuh"
 #include "fa_fwd_sm100.cuh"
@@ -142,7 +143,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   return check_launch("fa_fwd_sm100_kernel");
 }
 
-template <int D, bool WITH_DQ>
+template <int D>
 int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
                int B, int H, int H_kv, int N, float scale, int causal, const uint8_t* bm,
                const int32_t* kv_len, const BwdWs& ws, uint8_t* wsb, cudaStream_t stream) {
@@ -154,7 +155,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void
   if ((rc = make_map(&mk, k, B * H_kv, N, D, 128, "k")) != FA_OK) return rc;
   if ((rc = make_map(&mv, v, B * H_kv, N, D, 128, "v")) != FA_OK) return rc;
   if ((rc = make_map(&mdo, dO, BH, N, D, L::BM, "dO")) != FA_OK) return rc;
-  if ((rc = set_smem(fa::fa_bwd_sm100_kernel<D, WITH_DQ>, L::SMEM_ALLOC)) != FA_OK) return rc;
+  if ((rc = set_smem(fa::fa_bwd_sm100_kernel<D>, L::SMEM_ALLOC)) != FA_OK) return rc;
   fa::BwdParams p;
   p.block_mask = bm;
   p.kv_len = kv_len;
@@ -174,8 +175,46 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void
   p.causal = causal ? 1 : 0;
   const long long grid = static_cast<long long>(p.n_ktiles) * B * H_kv;  // one CTA per K/V tile
   if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
-  fa::fa_bwd_sm100_kernel<D, WITH_DQ><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
+  fa::fa_bwd_sm100_kernel<D><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
   return check_launch("fa_bwd_sm100_kernel");
+}
+
+// dK and dV only, scores double-buffered (fa_bwd_dkdv_sm100.cuh).
+template <int D>
+int launch_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, void* dk,
+                    void* dv, int B, int H, int H_kv, int N, float scale, int causal,
+                    const uint8_t* bm, const int32_t* kv_len, const BwdWs& ws, uint8_t* wsb,
+                    cudaStream_t stream) {
+  using L = fa::BwdDkdvLayout<D>;
+  CUtensorMap mq, mk, mv, mdo;
+  const int BH = B * H;
+  int rc;
+  if ((rc = make_map(&mq, q, BH, N, D, L::BM, "q")) != FA_OK) return rc;
+  if ((rc = make_map(&mk, k, B * H_kv, N, D, 128, "k")) != FA_OK) return rc;
+  if ((rc = make_map(&mv, v, B * H_kv, N, D, 128, "v")) != FA_OK) return rc;
+  if ((rc = make_map(&mdo, dO, BH, N, D, L::BM, "dO")) != FA_OK) return rc;
+  if ((rc = set_smem(fa::fa_bwd_dkdv_sm100_kernel<D>, L::SMEM_ALLOC)) != FA_OK) return rc;
+  fa::BwdParams p;
+  p.block_mask = bm;
+  p.kv_len = kv_len;
+  p.lse2 = reinterpret_cast<const float*>(wsb + ws.lse2);
+  p.dvec = reinterpret_cast<const float*>(wsb + ws.dvec);
+  p.dq_acc = nullptr;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.B = B;
+  p.H = H;
+  p.H_kv = H_kv;
+  p.N = N;
+  p.N_pad = ws.n_pad;
+  p.n_ktiles = (N + 127) / 128;
+  p.scale = scale;
+  p.scale2 = scale * kLog2e;
+  p.causal = causal ? 1 : 0;
+  const long long grid = static_cast<long long>(p.n_ktiles) * B * H_kv;
+  if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
+  fa::fa_bwd_dkdv_sm100_kernel<D><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
+  return check_launch("fa_bwd_dkdv_sm100_kernel");
 }
 
 // dQ without atomics: one CTA per 128 query rows walks the KV tiles (fa_bwd_dq_sm100.cuh).
@@ -319,18 +358,18 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   if (deterministic) {
     // dK and dV by the main kernel without its dQ part, dQ by the query-stationary kernel
     if (d == 64)
-      rc = launch_bwd<64, false>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+      rc = launch_bwd_dkdv<64>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
     else
-      rc = launch_bwd<128, false>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+      rc = launch_bwd_dkdv<128>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
     if (rc != FA_OK) return rc;
     if (d == 64)
       return launch_bwd_dq<64>(q, k, v, dO, dq, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
     return launch_bwd_dq<128>(q, k, v, dO, dq, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
   }
   if (d == 64)
-    rc = launch_bwd<64, true>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+    rc = launch_bwd<64>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
   else
-    rc = launch_bwd<128, true>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+    rc = launch_bwd<128>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
   if (rc != FA_OK) return rc;
   const long long n = static_cast<long long>(BH) * N * d;
   fa::dq_convert_kernel<<<static_cast<unsigned>((n / 8 + 255) / 256 + 1), 256, 0, s>>>(
@@ -533,9 +572,9 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
       reinterpret_cast<float*>(wsb + ws.dq), BH, N, ws.n_pad, d);
   if ((rc = check_launch("bwd_preprocess_kernel")) != FA_OK) return rc;
   if (d == 64)
-    rc = launch_bwd<64, true>(q, k, v, dO, dk, dv, B, H, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+    rc = launch_bwd<64>(q, k, v, dO, dk, dv, B, H, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
   else
-    rc = launch_bwd<128, true>(q, k, v, dO, dk, dv, B, H, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+    rc = launch_bwd<128>(q, k, v, dO, dk, dv, B, H, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
   if (rc != FA_OK) return rc;
   const long long n = static_cast<long long>(BH) * N * d;
   fa::dq_convert_kernel<<<static_cast<unsigned>((n / 8 + 255) / 256 + 1), 256, 0, s>>>(

@@ -95,9 +95,7 @@ enum : int {
   SITE_BWD_MMA_P = 33, SITE_BWD_C_DP = 34
 };
 
-// WITH_DQ = false: dK and dV only (the deterministic backward computes dQ in
-// fa_bwd_dq_sm100_kernel); the dS smem tile, the dQ MMA and the dQ warpgroup's work drop out.
-template <int D, bool WITH_DQ = true>
+template <int D>
 // 14 warps: some SM sub-partitions hold four of them, which caps registers at 128 per thread.
 __global__ void __launch_bounds__(448, 1)
 fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -339,16 +337,14 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           mma_scores(v_kd, do_kd, st1, L::DP_COL);
           mma_commit_w(bar_dp);
         }
-        if constexpr (WITH_DQ) {
-          if (t >= 2 &&
-              !mbar_wait_w(&bar_dqe[buf], ((t - 2) >> 1) & 1, abort_flag, SITE_BWD_MMA_DQE)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          mma_dq(buf);
-          mma_commit_w(&bar_dqf[buf]);
+        if (t >= 2 &&
+            !mbar_wait_w(&bar_dqe[buf], ((t - 2) >> 1) & 1, abort_flag, SITE_BWD_MMA_DQE)) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        mma_dq(buf);
+        mma_commit_w(&bar_dqf[buf]);
       }
       mma_commit_w(bar_done);
       mma_commit_w(bar_fin);
@@ -440,11 +436,10 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_arrive(bar_p);
       // ---- dS = P (dP - Dvec): bf16 into TMEM (over my dP^T) and into smem for the dQ MMA
       got = mbar_wait(bar_dp, t & 1, abort_flag, SITE_BWD_C_DP);
-      if (WITH_DQ && t >= 2)
-        got = got && mbar_wait(&bar_dqf[buf], ((t - 2) >> 1) & 1, abort_flag, SITE_BWD_C_DQ);
+      if (t >= 2) got = got && mbar_wait(&bar_dqf[buf], ((t - 2) >> 1) & 1, abort_flag, SITE_BWD_C_DQ);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
-      [[maybe_unused]] uint8_t* ds_row = smem + L::OFF_DS + buf * L::DS_TILE + jl * 128;
+      uint8_t* ds_row = smem + L::OFF_DS + buf * L::DS_TILE + jl * 128;
 #pragma unroll
       for (int c = 0; c < L::NCH; ++c) {
         uint32_t dr[32];
@@ -473,21 +468,19 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int i = 0; i < 16; ++i) dd[i] = pack_bf16x2(dsv[2 * i], dsv[2 * i + 1]);
         tmem_st16(dp_cols + 16 * c, dd);
-        if constexpr (WITH_DQ) {
-          // dS^T row jl, query columns c0+32c .. +31 -> 4 swizzled 16-byte chunks
-          const int col = c0 + 32 * c;
-          const int iblk = col >> 6;
-          const int chunk0 = (col & 63) >> 3;
+        // dS^T row jl, query columns c0+32c .. +31 -> 4 swizzled 16-byte chunks
+        const int col = c0 + 32 * c;
+        const int iblk = col >> 6;
+        const int chunk0 = (col & 63) >> 3;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int pos = (chunk0 + u) ^ (jl & 7);
-            *reinterpret_cast<uint4*>(ds_row + iblk * L::DS_IBLK + pos * 16) =
-                make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
-          }
+        for (int u = 0; u < 4; ++u) {
+          const int pos = (chunk0 + u) ^ (jl & 7);
+          *reinterpret_cast<uint4*>(ds_row + iblk * L::DS_IBLK + pos * 16) =
+              make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
         }
       }
       tmem_st_wait();
-      if constexpr (WITH_DQ) fence_proxy_async_smem();
+      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar_ds);
       ++t;
@@ -531,7 +524,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int qw = warp & 3;
     const uint32_t t_lane = static_cast<uint32_t>(32 * qw) << 16;
     int t = 0;
-    for (int w = 0; WITH_DQ && w < G * span; ++w) {
+    for (int w = 0; w < G * span; ++w) {
       const int g = w / span;
       const int it = it_first + (w - g * span);
       if (!q_active(it)) continue;

@@ -1,6 +1,6 @@
 """Deterministic backward on the GPU (fa_bwd_deterministic): dQ from the query-stationary
-tensor-core kernel without atomics, dK/dV from the main kernel without its dQ part.  Parity
-with the FP64 oracle, bit-identical repeats, and dK/dV bit-identical to fa_bwd's."""
+tensor-core kernel without atomics, dK/dV from the double-buffered dK/dV kernel.  Parity with
+the FP64 oracle, bit-identical repeats, and dV (and dK at d = 128) bit-identical to fa_bwd's."""
 import numpy as np
 import pytest
 import torch
@@ -50,9 +50,12 @@ def test_deterministic_backward_parity(cuda_lib, case):
     compare_grad(f64(dq), rq, "dQ")
     compare_grad(f64(dk), rk, "dK")
     compare_grad(f64(dv), rv, "dV")
-    # the main kernel without its dQ part computes dK and dV exactly as fa_bwd does
+    # the dK/dV kernel repeats fa_bwd's arithmetic: dV bit for bit; dK too at d = 128, where
+    # both keep P in fp32 for dS (fa_bwd's d = 64 kernel reuses the bf16-rounded P there)
     _, dk2, dv2 = _run(cuda_lib, g, False)
-    assert torch.equal(dk, dk2) and torch.equal(dv, dv2)
+    assert torch.equal(dv, dv2)
+    if d == 128:
+        assert torch.equal(dk, dk2)
 
 
 def test_deterministic_backward_repeats_bit_identically(cuda_lib):
