@@ -306,11 +306,10 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   return fail(FA_ERR_INVALID, "unknown dtype %d", dtype);
 }
 
-int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse,
-             const void* dO, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
-             float scale, int causal, const uint8_t* block_mask, const int32_t* kv_len,
-             int dtype, void* workspace, size_t workspace_bytes, void* stream,
-             bool deterministic) {
+// Argument checks shared by every backward entry point (everything but the workspace).
+int bwd_checks(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dO, const void* dq, const void* dk, const void* dv, int B, int H,
+               int H_kv, int N, int d, float scale, int dtype) {
   int rc = common_checks(q, k, v, o, lse, B, H, N, d, scale);
   if (rc != FA_OK) return rc;
   if ((rc = check_groups(H, H_kv)) != FA_OK) return rc;
@@ -322,6 +321,16 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     return fail(FA_ERR_UNSUPPORTED, "fp32 backward supports d <= 128, got %d", d);
   if (dtype == FA_BF16 && d != 64 && d != 128)
     return fail(FA_ERR_UNSUPPORTED, "bf16 backward supports d in {64, 128}, got %d", d);
+  return FA_OK;
+}
+
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* dO, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
+             float scale, int causal, const uint8_t* block_mask, const int32_t* kv_len,
+             int dtype, void* workspace, size_t workspace_bytes, void* stream,
+             bool deterministic) {
+  int rc = bwd_checks(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, scale, dtype);
+  if (rc != FA_OK) return rc;
   const BwdWs ws = bwd_ws(B, H, N, d);
   if (workspace == nullptr || workspace_bytes < ws.total)
     return fail(FA_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", ws.total, workspace_bytes);
@@ -541,17 +550,8 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
                               int B, int H, int N, int d, float scale, int causal,
                               const uint8_t* block_mask, const int32_t* kv_len, int dtype,
                               void* stream) {
-  int rc = common_checks(q, k, v, o, lse, B, H, N, d, scale);
+  int rc = bwd_checks(q, k, v, o, lse, dO, dq, dk, dv, B, H, H, N, d, scale, dtype);
   if (rc != FA_OK) return rc;
-  if (!dO || !dq || !dk || !dv) return fail(FA_ERR_INVALID, "null gradient pointer");
-  if (!aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
-    return fail(FA_ERR_ALIGN, "gradient pointers must be 16-byte aligned");
-  if (dtype != FA_BF16) {
-    if (dtype == FA_F32) return fail(FA_ERR_UNSUPPORTED, "fp32 backward is not built");
-    return fail(FA_ERR_INVALID, "unknown dtype %d", dtype);
-  }
-  if (d != 64 && d != 128)
-    return fail(FA_ERR_UNSUPPORTED, "bf16 backward supports d in {64, 128}, got %d", d);
   const BwdWs ws = bwd_ws(B, H, N, d);
   if (ws.total > kNoAllocScratchBytes)
     return fail(FA_ERR_WORKSPACE,
@@ -560,24 +560,8 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
                 ws.total, kNoAllocScratchBytes);
   void* scratch = nullptr;
   if ((rc = noalloc_scratch(&scratch)) != FA_OK) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* wsb = static_cast<uint8_t*>(scratch);
-  const int BH = B * H;
-  // The preprocess kernel rewrites lse2 / Dvec and zeroes the dQ accumulator, so whatever the
-  // previous call left in the scratch never leaks into this one.
-  const long long pre_rows = static_cast<long long>(BH) * ws.n_pad;
-  fa::bwd_preprocess_kernel<<<static_cast<unsigned>((pre_rows + 7) / 8), 256, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse,
-      reinterpret_cast<float*>(wsb + ws.lse2), reinterpret_cast<float*>(wsb + ws.dvec),
-      reinterpret_cast<float*>(wsb + ws.dq), BH, N, ws.n_pad, d);
-  if ((rc = check_launch("bwd_preprocess_kernel")) != FA_OK) return rc;
-  if (d == 64)
-    rc = launch_bwd<64>(q, k, v, dO, dk, dv, B, H, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
-  else
-    rc = launch_bwd<128>(q, k, v, dO, dk, dv, B, H, H, N, scale, causal, block_mask, kv_len, ws, wsb, s);
-  if (rc != FA_OK) return rc;
-  const long long n = static_cast<long long>(BH) * N * d;
-  fa::dq_convert_kernel<<<static_cast<unsigned>((n / 8 + 255) / 256 + 1), 256, 0, s>>>(
-      reinterpret_cast<const float*>(wsb + ws.dq), static_cast<__nv_bfloat16*>(dq), n, scale);
-  return check_launch("dq_convert_kernel");
+  // fa_bwd's path on the built-in scratch.  Its first kernel rewrites lse2 / Dvec and zeroes the
+  // dQ accumulator, so whatever the previous call left in the scratch never leaks into this one.
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, H, N, d, scale, causal, block_mask,
+                  kv_len, dtype, scratch, kNoAllocScratchBytes, stream, false);
 }

@@ -20,18 +20,19 @@ import synthetic as syn
 from gpu_util import compare_grad, f64, to_gpu
 
 CASES = [
-    # B, H, N, d, causal, kv_len, block mask
-    (2, 3, 700, 64, True, None, False),
-    (1, 2, 1000, 128, False, [1000], False),
-    (3, 2, 512, 64, False, [130, 512, 301], True),
+    # B, H, N, d, causal, kv_len, block mask, dtype
+    (2, 3, 700, 64, True, None, False, "bf16"),
+    (1, 2, 1000, 128, False, [1000], False, "bf16"),
+    (3, 2, 512, 64, False, [130, 512, 301], True, "bf16"),
+    (1, 2, 300, 100, True, None, False, "f32"),  # the fp32 backward on the same scratch
 ]
 
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("case", range(len(CASES)))
 def test_noalloc_matches_workspace_backward(cuda_lib, case):
-    B, H, N, d, causal, L, use_bm = CASES[case]
-    x = syn.make_inputs(B, H, N, d, "bf16", seed=3100 + case, causal=causal,
+    B, H, N, d, causal, L, use_bm, dt = CASES[case]
+    x = syn.make_inputs(B, H, N, d, dt, seed=3100 + case, causal=causal,
                         kv_len=None if L is None else np.array(L, np.int32),
                         block_mask=syn.block_mask_band_global(N) if use_bm else None)
     g = to_gpu(x)
