@@ -53,7 +53,7 @@ template <int D>
 struct BwdLayout {
   static constexpr int BN = 128;                  // keys per CTA
   static constexpr int BM = D == 64 ? 128 : 64;   // query rows per step
-  static constexpr int QST = 3;                   // Q/dO/lse/Dvec stages
+  static constexpr int QST = D == 128 ? 4 : 3;    // Q/dO/lse/Dvec stages
   static constexpr int SUB = D / 64;
   static constexpr int KV_SUBTILE = 128 * 128;
   static constexpr int Q_SUBTILE = BM * 128;
@@ -78,7 +78,10 @@ struct BwdLayout {
   static constexpr int EMU_EVERY = 0;               // one P pair in EMU_EVERY exponentiated on FMA (0: none)
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
-  static constexpr int SMEM_ALLOC = BYTES + 1024;
+  // Dynamic shared memory starts 1024-byte aligned on sm_100 (the kernel checks), so no slack
+  // is allocated: at d = 128 the fourth Q/dO stage fits only without it.
+  static constexpr int SMEM_ALLOC = BYTES;
+  static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL = 0;
   static constexpr uint32_t DP_COL = BM;
@@ -92,7 +95,7 @@ enum : int {
   SITE_BWD_LOAD_EMPTY = 21, SITE_BWD_LOAD_DRAIN = 22, SITE_BWD_MMA_KV = 23, SITE_BWD_MMA_Q = 24,
   SITE_BWD_MMA_DS = 25, SITE_BWD_MMA_DQE = 26, SITE_BWD_MMA_FIN = 27, SITE_BWD_C_Q = 28,
   SITE_BWD_C_S = 29, SITE_BWD_C_DQ = 30, SITE_BWD_C_DONE = 31, SITE_BWD_DQ = 32,
-  SITE_BWD_MMA_P = 33, SITE_BWD_C_DP = 34
+  SITE_BWD_MMA_P = 33, SITE_BWD_C_DP = 34, SITE_BWD_SMEM_ALIGN = 35
 };
 
 template <int D>
@@ -104,9 +107,15 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
   using L = BwdLayout<D>;
   constexpr int BM = L::BM;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 128-byte-swizzled TMA tiles need 1024-byte alignment; without slack in the allocation a
+  // misaligned base is reported (status word) and the CTA returns before touching anything.
+  if ((smem_u32(smem_raw) & 1023u) != 0u) {
+    if (threadIdx.x == 0)
+      atomicCAS(&g_status, 0u, (static_cast<unsigned>(SITE_BWD_SMEM_ALIGN) << 16) | (blockIdx.x & 0xffffu));
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* bar_kv = bars;
   uint64_t* bar_qf = bars + 1;
