@@ -365,7 +365,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
       deterministic ? nullptr : reinterpret_cast<float*>(wsb + ws.dq), BH, N, ws.n_pad, d);
   if ((rc = check_launch("bwd_preprocess_kernel")) != FA_OK) return rc;
   if (deterministic) {
-    // dK and dV by the main kernel without its dQ part, dQ by the query-stationary kernel
+    // dK and dV by the dK/dV kernel, dQ by the query-stationary kernel: no atomics
     if (d == 64)
       rc = launch_bwd_dkdv<64>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
     else
