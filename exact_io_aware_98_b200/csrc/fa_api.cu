@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -173,6 +174,13 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void
   p.scale = scale;
   p.scale2 = scale * kLog2e;
   p.causal = causal ? 1 : 0;
+  {
+    // K/V heads per CTA-order group: the group's dQ accumulator (fp32), Q and dO, 8 bytes per
+    // element of its G query heads, within half of the 126 MB L2.
+    const long long per_head = 8ll * (H / H_kv) * N * D;
+    const long long fit = (64ll << 20) / per_head;
+    p.hgroup = static_cast<int>(std::max(1ll, std::min(fit, static_cast<long long>(B) * H_kv)));
+  }
   const long long grid = static_cast<long long>(p.n_ktiles) * B * H_kv;  // one CTA per K/V tile
   if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
   fa::fa_bwd_sm100_kernel<D><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
@@ -200,6 +208,7 @@ int launch_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
   p.lse2 = reinterpret_cast<const float*>(wsb + ws.lse2);
   p.dvec = reinterpret_cast<const float*>(wsb + ws.dvec);
   p.dq_acc = nullptr;
+  p.hgroup = B * H_kv;                                   // not read by the dK/dV kernel
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.B = B;

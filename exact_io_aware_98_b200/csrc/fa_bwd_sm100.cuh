@@ -45,6 +45,7 @@ struct BwdParams {
   int B, H, N, N_pad;
   int H_kv;                   // K/V heads: query heads G*j .. G*j+G-1 (G = H / H_kv) read head j
   int n_ktiles;               // ceil(N / 128)
+  int hgroup;                 // K/V heads per CTA-order group (>= 1; B*H_kv: one group)
   float scale, scale2;
   int causal;
 };
@@ -137,8 +138,16 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int lane = threadIdx.x & 31;
   const int G = p.H / p.H_kv;                         // query heads per K/V head
   const int BHkv = p.B * p.H_kv;
-  const int jt = static_cast<int>(blockIdx.x) / BHkv;  // KV tile; small jt (most work) first
-  const int bhk = static_cast<int>(blockIdx.x) % BHkv;  // (b, K/V head)
+  // CTA order: groups of p.hgroup K/V heads in turn, and inside a group the KV tiles with the
+  // most query tiles (small jt) first.  A group's fp32 dQ accumulator, Q and dO fit in L2, so
+  // the dQ reductions of the CTAs in flight hit L2 instead of missing to HBM.
+  const int per_group = p.hgroup * p.n_ktiles;
+  const int grp = static_cast<int>(blockIdx.x) / per_group;
+  const int g0 = grp * p.hgroup;
+  const int gn = min(p.hgroup, BHkv - g0);             // heads in this group (the last may have fewer)
+  const int r = static_cast<int>(blockIdx.x) - grp * per_group;
+  const int jt = r / gn;                               // KV tile
+  const int bhk = g0 + r % gn;                         // (b, K/V head)
   const int b = bhk / p.H_kv;
   const int bhq0 = b * p.H + (bhk % p.H_kv) * G;       // first query head of the group
   const int N = p.N;
