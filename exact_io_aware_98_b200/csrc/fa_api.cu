@@ -75,6 +75,24 @@ int make_map(CUtensorMap* map, const void* base, int BH, int N, int d, int box_r
   return FA_OK;
 }
 
+// 3-D view [B*H][N][d] of the fp32 dQ accumulator for TMA reduce-adds: unswizzled boxes of
+// 32 columns x 64 rows.
+int make_dq_map(CUtensorMap* map, float* base, int BH, int N, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4,
+                                 static_cast<cuuint64_t>(N) * d * 4};
+  const cuuint32_t box[3] = {32u, 64u, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "tensor map for the dQ accumulator failed (%d)", (int)r);
+  return FA_OK;
+}
+
 template <typename Kernel>
 int set_smem(Kernel kernel, int bytes) {
   const cudaError_t e =
@@ -149,13 +167,18 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void
                int B, int H, int H_kv, int N, float scale, int causal, const uint8_t* bm,
                const int32_t* kv_len, const BwdWs& ws, uint8_t* wsb, cudaStream_t stream) {
   using L = fa::BwdLayout<D>;
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   const int BH = B * H;
   int rc;
   if ((rc = make_map(&mq, q, BH, N, D, L::BM, "q")) != FA_OK) return rc;
   if ((rc = make_map(&mk, k, B * H_kv, N, D, 128, "k")) != FA_OK) return rc;
   if ((rc = make_map(&mv, v, B * H_kv, N, D, 128, "v")) != FA_OK) return rc;
   if ((rc = make_map(&mdo, dO, BH, N, D, L::BM, "dO")) != FA_OK) return rc;
+  if (L::V_IN_TMEM) {
+    if ((rc = make_dq_map(&mdq, reinterpret_cast<float*>(wsb + ws.dq), BH, N, D)) != FA_OK) return rc;
+  } else {
+    mdq = mq;  // not read at d = 64 (dQ by vector atomics)
+  }
   if ((rc = set_smem(fa::fa_bwd_sm100_kernel<D>, L::SMEM_ALLOC)) != FA_OK) return rc;
   fa::BwdParams p;
   p.block_mask = bm;
@@ -183,7 +206,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void
   }
   const long long grid = static_cast<long long>(p.n_ktiles) * B * H_kv;  // one CTA per K/V tile
   if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
-  fa::fa_bwd_sm100_kernel<D><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
+  fa::fa_bwd_sm100_kernel<D><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, mdq, p);
   return check_launch("fa_bwd_sm100_kernel");
 }
 

@@ -14,14 +14,18 @@
 // One CTA owns 128 keys (K and V stay in shared memory) and walks the query tiles that can
 // see them (causal, key padding and block mask skip whole tiles).  Per query tile of BM rows:
 //   S^T  = K Q^T     (M=128 keys, N=BM, K=D)      smem x smem  -> TMEM
-//   dP^T = V dO^T    (M=128, N=BM, K=D)           smem x smem  -> TMEM
+//   dP^T = V dO^T    (M=128, N=BM, K=D)           smem x smem  -> TMEM (D=64)
+//                                                 TMEM x smem  -> TMEM (D=128: V copied
+//                                                 into TMEM once per CTA)
 //   compute warpgroups (two, each owning half of the BM query columns): P^T and dS^T in bf16
 //   back into TMEM (each over the front half of its own S^T / dP^T columns) and dS^T to smem
 //   dV  += P^T dO    (M=128, N=D, K=BM)           TMEM x smem  -> TMEM
 //   dK  += dS^T Q    (M=128, N=D, K=BM)           TMEM x smem  -> TMEM
 //   D=64 : dQ   = dS K     (M=BM=128, N=64,  K=128) smem x smem -> TMEM (row per lane)
 //   D=128: dQ^T = K^T dS^T (M=128,    N=BM=64, K=128) smem x smem -> TMEM (column per lane)
-//   dQ warpgroup: TMEM -> fp32 red.global.add into the dQ workspace.
+//   dQ warpgroup: TMEM -> the fp32 dQ workspace, by vector red.global.add at D=64 and at
+//   D=128 by one TMA reduce-add per warp of a [64 rows][32 d] box staged in the V tile's
+//   shared memory (free once V is in TMEM).
 // Hand-offs per step: P ready (-> dV(t), then S(t+1)) and dS ready (-> dK(t), then dP(t+1),
 // then dQ(t)).  In-order MMA execution lets S(t+1) reuse the TMEM that dV(t) read P^T(t) from,
 // and dP(t+1) the TMEM of dS^T(t); the compute warpgroups compute dS(t) while dV(t) and S(t+1)
@@ -71,8 +75,8 @@ struct BwdLayout {
   static constexpr int OFF_DVEC = OFF_LSE + QST * BM * 4;
   static constexpr int OFF_BAR = OFF_DVEC + QST * BM * 4;
   // kv, q_full[QST], q_empty[QST], s_full, dp_full, p_full, ds_full, dq_full[2], dq_empty[2],
-  // kv_done, fin
-  static constexpr int NBAR = 1 + 2 * QST + 4 + 2 + 2 + 1 + 1;
+  // kv_done, fin, v_tmem
+  static constexpr int NBAR = 1 + 2 * QST + 4 + 2 + 2 + 1 + 1 + 1;
   static constexpr int THREADS = 448;
   static constexpr int HALF = BM / 2;               // query columns per compute warpgroup
   static constexpr int NCH = HALF / 32;             // 32-column chunks per compute warpgroup
@@ -84,11 +88,20 @@ struct BwdLayout {
   static constexpr int SMEM_ALLOC = BYTES;
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
   static constexpr uint32_t TMEM_COLS = 512;
+  // d = 128: V moves into TMEM (the A operand of dP^T) once per CTA, and its shared-memory tile
+  // then stages dQ^T for TMA reduce-adds into the fp32 accumulator (no per-element atomics).
+  // The 64 TMEM columns come from holding one dQ^T buffer instead of two.
+  static constexpr bool V_IN_TMEM = D == 128;
+  static constexpr int DQB = V_IN_TMEM ? 1 : 2;         // dQ buffers of 64 columns
   static constexpr uint32_t S_COL = 0;
   static constexpr uint32_t DP_COL = BM;
-  static constexpr uint32_t DQ_COL = 2 * BM;           // two 64-column buffers
+  static constexpr uint32_t DQ_COL = 2 * BM;
+  static constexpr uint32_t VT_COL = DQ_COL + DQB * 64;  // V, d = 128 only
   static constexpr uint32_t DV_COL = 2 * BM + 128;
   static constexpr uint32_t DK_COL = 2 * BM + 128 + D;
+  static_assert(!V_IN_TMEM || VT_COL + D / 2 <= DV_COL, "TMEM: V overlaps dV");
+  static constexpr int DQ_STAGE = 64 * 32 * 4;         // one dQ warp's [64 rows][32 d] fp32 box
+  static_assert(!V_IN_TMEM || 4 * DQ_STAGE <= KV_TILE, "dQ staging fits in the V tile");
   static_assert(DK_COL + D <= TMEM_COLS, "TMEM budget");
 };
 
@@ -96,16 +109,19 @@ enum : int {
   SITE_BWD_LOAD_EMPTY = 21, SITE_BWD_LOAD_DRAIN = 22, SITE_BWD_MMA_KV = 23, SITE_BWD_MMA_Q = 24,
   SITE_BWD_MMA_DS = 25, SITE_BWD_MMA_DQE = 26, SITE_BWD_MMA_FIN = 27, SITE_BWD_C_Q = 28,
   SITE_BWD_C_S = 29, SITE_BWD_C_DQ = 30, SITE_BWD_C_DONE = 31, SITE_BWD_DQ = 32,
-  SITE_BWD_MMA_P = 33, SITE_BWD_C_DP = 34, SITE_BWD_SMEM_ALIGN = 35
+  SITE_BWD_MMA_P = 33, SITE_BWD_C_DP = 34, SITE_BWD_SMEM_ALIGN = 35, SITE_BWD_MMA_VT = 36,
+  SITE_BWD_C_KV = 37
 };
 
 template <int D>
 // 14 warps: some SM sub-partitions hold four of them, which caps registers at 128 per thread.
+// tm_dq: the fp32 dQ accumulator [B*H][N][D], boxes of 32 columns x 64 rows (d = 128 only).
 __global__ void __launch_bounds__(448, 1)
 fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
-                    const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using L = BwdLayout<D>;
   constexpr int BM = L::BM;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -129,6 +145,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint64_t* bar_dqe = bar_dqf + 2;
   uint64_t* bar_done = bar_dqe + 2;
   uint64_t* bar_fin = bar_done + 1;
+  uint64_t* bar_vt = bar_fin + 1;        // V copied into TMEM (d = 128)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
   const float* s_lse = reinterpret_cast<const float*>(smem + L::OFF_LSE);
@@ -194,6 +211,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     mbar_init(bar_done, 1);
     mbar_init(bar_fin, 1);
+    mbar_init(bar_vt, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -269,18 +287,31 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint64_t ds_mn = sdesc_sw128(ds_addr, L::DS_IBLK, 1024);
       auto off16 = [](int bytes) -> uint64_t { return static_cast<uint64_t>(bytes >> 4); };
       // X^T = A B^T over D: A = K or V (128 rows), B = Q or dO of stage st (BM rows), K-major.
-      auto mma_scores = [&](uint64_t a_desc, uint64_t b_desc, int st, uint32_t d_col) {
+      // a_tmem: A is V in TMEM (16 elements of d per K-step = 8 columns).
+      auto mma_scores = [&](uint64_t a_desc, bool a_tmem, uint64_t b_desc, int st, uint32_t d_col) {
         const uint64_t bst = b_desc + off16(st * L::Q_TILE);
 #pragma unroll
         for (int kb = 0; kb < D / 64; ++kb) {
-          uint64_t a[4], b[4];
+          uint64_t b[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int k = 4 * kb + i;
-            a[i] = a_desc + off16((k >> 2) * L::KV_SUBTILE + (k & 3) * 32);
             b[i] = bst + off16((k >> 2) * L::Q_SUBTILE + (k & 3) * 32);
           }
-          mma_ss_x4(tmem + d_col, a, b, idesc_s, kb > 0 ? 1u : 0u);
+          if (a_tmem) {
+            uint32_t a[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = tmem + L::VT_COL + 8u * (4 * kb + i);
+            mma_ts_x4(tmem + d_col, a, b, idesc_s, kb > 0 ? 1u : 0u);
+          } else {
+            uint64_t a[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int k = 4 * kb + i;
+              a[i] = a_desc + off16((k >> 2) * L::KV_SUBTILE + (k & 3) * 32);
+            }
+            mma_ss_x4(tmem + d_col, a, b, idesc_s, kb > 0 ? 1u : 0u);
+          }
         }
       };
       // G += X^T(TMEM, bf16) B over BM rows: B = dO or Q of stage st, MN-major.  Query columns
@@ -318,16 +349,22 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
               b[i] = ds + off16(k * 2048);
             }
           }
-          mma_ss_x4(tmem + L::DQ_COL + buf * 64, a, b, idesc_q, kb > 0 ? 1u : 0u);
+          mma_ss_x4(tmem + L::DQ_COL + (buf % L::DQB) * 64, a, b, idesc_q, kb > 0 ? 1u : 0u);
         }
       };
       bool ok = mbar_wait_w(bar_kv, 0, abort_flag, SITE_BWD_MMA_KV);
       ok = ok && mbar_wait_w(&bar_qf[0], 0, abort_flag, SITE_BWD_MMA_Q);
       tc_fence_after();
       if (ok) {
-        mma_scores(k_kd, q_kd, 0, L::S_COL);
+        mma_scores(k_kd, false, q_kd, 0, L::S_COL);
         mma_commit_w(bar_s);
-        mma_scores(v_kd, do_kd, 0, L::DP_COL);
+        if (L::V_IN_TMEM) {
+          ok = mbar_wait_w(bar_vt, 0, abort_flag, SITE_BWD_MMA_VT);
+          tc_fence_after();
+        }
+      }
+      if (ok) {
+        mma_scores(v_kd, L::V_IN_TMEM, do_kd, 0, L::DP_COL);
         mma_commit_w(bar_dp);
       }
       for (int t = 0; ok && t < n_steps; ++t) {
@@ -344,7 +381,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             break;
           }
           tc_fence_after();
-          mma_scores(k_kd, q_kd, st1, L::S_COL);
+          mma_scores(k_kd, false, q_kd, st1, L::S_COL);
           mma_commit_w(bar_s);
         }
         if (!mbar_wait_w(bar_ds, t & 1, abort_flag, SITE_BWD_MMA_DS)) { ok = false; break; }
@@ -352,11 +389,12 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         mma_grad(L::DP_COL, q_mn, st, L::DK_COL, t > 0);
         mma_commit_w(&bar_qe[st]);  // Q(t), dO(t), lse(t), Dvec(t) are no longer read after dK(t)
         if (next) {
-          mma_scores(v_kd, do_kd, st1, L::DP_COL);
+          mma_scores(v_kd, L::V_IN_TMEM, do_kd, st1, L::DP_COL);
           mma_commit_w(bar_dp);
         }
-        if (t >= 2 &&
-            !mbar_wait_w(&bar_dqe[buf], ((t - 2) >> 1) & 1, abort_flag, SITE_BWD_MMA_DQE)) {
+        // dQ(t) into TMEM buffer t % DQB once dQ(t - DQB) has been read out of it
+        if (t >= L::DQB && !mbar_wait_w(&bar_dqe[(t - L::DQB) & 1], ((t - L::DQB) >> 1) & 1,
+                                        abort_flag, SITE_BWD_MMA_DQE)) {
           ok = false;
           break;
         }
@@ -379,8 +417,33 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t dp_cols = tmem + t_lane + L::DP_COL + h * L::HALF;  // my dP^T columns
     const float scale2 = p.scale2;
     bool ok = true;
+    if (L::V_IN_TMEM && h == 0 && n_steps > 0) {
+      // V row jl into TMEM as the A operand of dP^T: 16-byte chunk c of sub-tile s holds
+      // d = 64s + 8c .. +7 at swizzled position c ^ (jl & 7); a column holds a pair of d.
+      const bool got = mbar_wait(bar_kv, 0, abort_flag, SITE_BWD_C_KV);
+      ok = __all_sync(0xffffffffu, got);
+      if (ok) {
+#pragma unroll
+        for (int s = 0; s < L::SUB; ++s) {
+          uint32_t vr[32];
+          const uint8_t* vrow = smem + L::OFF_V + s * L::KV_SUBTILE + jl * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v4 = *reinterpret_cast<const uint4*>(vrow + ((c ^ (jl & 7)) * 16));
+            vr[4 * c] = v4.x;
+            vr[4 * c + 1] = v4.y;
+            vr[4 * c + 2] = v4.z;
+            vr[4 * c + 3] = v4.w;
+          }
+          tmem_st32(tmem + t_lane + L::VT_COL + 32 * s, vr);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+      }
+      mbar_arrive(bar_vt);
+    }
     int t = 0;
-    for (int w = 0; w < G * span; ++w) {
+    for (int w = 0; ok && w < G * span; ++w) {
       const int g = w / span;
       const int it = it_first + (w - g * span);
       if (!q_active(it)) continue;
@@ -553,8 +616,8 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       uint32_t v[2][32];
-      tmem_ld32(tmem + t_lane + L::DQ_COL + buf * 64, v[0]);
-      tmem_ld32(tmem + t_lane + L::DQ_COL + buf * 64 + 32, v[1]);
+      tmem_ld32(tmem + t_lane + L::DQ_COL + (buf % L::DQB) * 64, v[0]);
+      tmem_ld32(tmem + t_lane + L::DQ_COL + (buf % L::DQB) * 64 + 32, v[1]);
       tmem_ld_wait();
       reg_fence(v[0]);
       reg_fence(v[1]);
@@ -573,15 +636,28 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
         }
       } else {
-        // lane = head dimension c, columns = query rows i0 .. i0+63
-        const int c = 32 * qw + lane;
-        float* base = p.dq_acc + (static_cast<size_t>(bh) * N + i0) * D + c;
+        // lane = head dimension 32qw + lane, columns = query rows i0 .. i0+63: staged as this
+        // warp's [64][32] fp32 box in the V tile (V lives in TMEM by now: dQ(0) follows the
+        // copy) and added to the accumulator by one TMA reduce (rows >= N are skipped).
+        float* stg = reinterpret_cast<float*>(smem + L::OFF_V + qw * L::DQ_STAGE);
+        if (t > 0) {
+          if (lane == 0) bulk_wait_read_all();  // the previous box has been read
+          __syncwarp();
+        }
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          if (i0 + i < N) atomicAdd(base + static_cast<size_t>(i) * D, __uint_as_float(v[i >> 5][i & 31]));
+        for (int i = 0; i < 64; ++i) stg[i * 32 + lane] = __uint_as_float(v[i >> 5][i & 31]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(&tm_dq, stg, 32 * qw, i0, bh);
+          bulk_commit_group();
         }
       }
       ++t;
+    }
+    if (L::V_IN_TMEM) {
+      if (lane == 0) bulk_wait_all();  // the reductions are complete before the CTA ends
+      __syncwarp();
     }
   }
 

@@ -75,7 +75,8 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  * fa_bwd -- backward pass of fa_fwd from (q, k, v, o, lse, dO), recomputing the scores:
  *   dV = A^T dO,  dS = A o (dO V^T - rowsum(dO o O)),  dQ = scale dS K,  dK = scale dS^T Q.
  *   dtype FA_BF16: d in {64, 128}; tensor-core kernel.  dq accumulates across key tiles with
- *                  fp32 atomics, so its last bits may differ between runs; dk and dv are
+ *                  fp32 reductions in L2 (atomics at d = 64, TMA reduce-adds at d = 128) whose
+ *                  order varies, so its last bits may differ between runs; dk and dv are
  *                  deterministic.
  *   dtype FA_F32 : 1 <= d <= 128; CUDA-core fp32 kernels (one warp per query row for dq, one
  *                  per key row for dk and dv), exact expf, every sum in a fixed order: all
