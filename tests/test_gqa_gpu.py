@@ -109,6 +109,33 @@ def test_gqa_llama_like_sampled(cuda_lib):
             compare_grad(f64(dq[0, h]), rq[0, h], f"dQ[{h}]")
 
 
+def test_gqa_long_all_groups(cuda_lib):
+    """B1 H32 H_kv8 N8192 d128 causal: the backward's CTAs run in groups of two K/V heads.  dK and
+    dV of every K/V head equal the deterministic backward's bit for bit, and dQ rows sampled over
+    all 32 query heads match the oracle (on K/V repeated per query head)."""
+    fa = cuda_lib
+    x = _inputs(1, 32, 8, 8192, 128, True, seed=1304)
+    g = to_gpu(x)
+    o, lse = _fwd(fa, g)
+    args = (g["q"], g["k"], g["v"], o, lse, g["do"], g["scale"], g["causal"], g["block_mask"],
+            g["kv_len"])
+    dq, dk, dv = fa.bwd(*args)
+    _, dk2, dv2 = fa.bwd(*args, deterministic=True)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    assert torch.equal(dk, dk2) and torch.equal(dv, dv2)
+    N = 8192
+    rows = np.unique(np.concatenate([np.random.default_rng(4).choice(32 * N, 200, replace=False),
+                                     [0, N - 1, 31 * N, 32 * N - 1]]))
+    rep = lambda t: np.repeat(f64(t), 4, axis=1)
+    rq = oracle.attn_bwd_dq_rows(f64(x["q"]), rep(x["k"]), rep(x["v"]), f64(x["do"]), x["scale"],
+                                 rows, True)
+    got = f64(dq).reshape(-1, 128)[rows]
+    scale = np.abs(rq).max()
+    assert np.abs(got - rq).max() / scale <= 2e-2
+    assert np.abs(got - rq).mean() / scale <= 2e-3
+
+
 def test_gqa_dkdv_deterministic(cuda_lib):
     g = to_gpu(_inputs(1, 6, 2, 640, 64, True, seed=1303))
     _, _, _, dk1, dv1 = _fb(cuda_lib, g)
