@@ -179,6 +179,32 @@ def max_over_ranks(values, dist, device) -> list:
     return [float(v) for v in t.tolist()]
 
 
+# MUFU (special-function unit) throughput for ex2: 16 results per clock per SM, the nominal
+# figure for recent NVIDIA architectures; 148 SMs on a B200.
+MUFU_PER_CLK_PER_SM = 16
+N_SM = 148
+
+
+def step_stats(ms: list) -> dict:
+    """Median and p10/p90 of per-step durations (the mean is reported beside them)."""
+    if len(ms) < 2:
+        return {"median_ms": round(ms[0], 4)} if ms else {}
+    q = statistics.quantiles(ms, n=10, method="inclusive")
+    return {"median_ms": round(statistics.median(ms), 4), "p10_ms": round(q[0], 4),
+            "p90_ms": round(q[-1], 4)}
+
+
+def exp_roof(pairs: float, ms: float, sm_mhz) -> dict:
+    """The second roof of both passes: one exponential per unmasked (query, key) pair, against
+    the MUFU ex2 rate at the sampled SM clock.  The forward takes part of its exponentials on
+    the FMA pipe, so its fraction can read above what MUFU alone could deliver."""
+    mhz = float(sm_mhz) if sm_mhz else 1965.0
+    peak = MUFU_PER_CLK_PER_SM * N_SM * mhz * 1e6
+    rate = pairs / (ms * 1e-3)
+    return {"exp_per_s": float("%.4g" % rate), "mufu_peak_per_s": float("%.4g" % peak),
+            "frac": round(rate / peak, 4), "sm_mhz": mhz}
+
+
 def aggregate_tflops(flop_per_rank_step: float, world: int, ms_per_step: float) -> float:
     """Whole-job throughput under weak scaling: every rank does one replica's work per step."""
     return flop_per_rank_step * world / (ms_per_step * 1e-3) / 1e12
@@ -234,8 +260,9 @@ def run_ours(args, rank: int, world: int, dist):
     if dist is not None:
         dist.barrier()
     total_ms = ev[0][0].elapsed_time(ev[K - 1][2])
-    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    fwd_all = [e[0].elapsed_time(e[1]) for e in ev]
+    bwd_all = [e[1].elapsed_time(e[2]) for e in ev]
+    fwd_ms, bwd_ms = statistics.mean(fwd_all), statistics.mean(bwd_all)
     total_ms, fwd_ms, bwd_ms = max_over_ranks([total_ms, fwd_ms, bwd_ms], dist, dev)
     status = fa.device_status()
 
@@ -283,9 +310,11 @@ def run_ours(args, rank: int, world: int, dist):
                    "l2": "inputs larger than L2: Q,K,V,dO are 4 x %.0f MiB per step"
                          % (x["q"].numel() * 2 / 2**20)},
         "fwd": {"ms": round(fwd_ms, 4), "tflops": round(fwd_tf, 2),
-                "frac_sustained": round(fwd_tf / sustained, 4)},
+                "frac_sustained": round(fwd_tf / sustained, 4), **step_stats(fwd_all),
+                "exp_roof": exp_roof(f_fwd / (4.0 * d), fwd_ms, clocks.get("sm_mhz"))},
         "bwd": {"ms": round(bwd_ms, 4), "tflops": round(bwd_tf, 2),
-                "frac_sustained": round(bwd_tf / sustained, 4)},
+                "frac_sustained": round(bwd_tf / sustained, 4), **step_stats(bwd_all),
+                "exp_roof": exp_roof(f_bwd / (10.0 * d), bwd_ms, clocks.get("sm_mhz"))},
         "roofline": roof,
         "clocks": clocks,
         # per step: fa_fwd's kernel + preprocess, main backward and dQ convert (or dQ kernel)
