@@ -154,6 +154,10 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.H_kv = H_kv;
   p.N = N;
   p.n_mtiles = (N + 255) / 256;
+  // Query heads per CTA-order group: Q, K, V and O of the group (8 bytes per element of each
+  // query head, K and V counted per query head) within half of the 126 MB L2.
+  p.hgroup = static_cast<int>(
+      std::max(1ll, std::min((64ll << 20) / (8ll * N * D), static_cast<long long>(BH))));
   p.scale2 = scale * kLog2e;
   p.causal = causal ? 1 : 0;
   const long long grid = static_cast<long long>(p.n_mtiles) * BH;

@@ -45,6 +45,7 @@ struct FwdParams {
   int B, H, N;
   int H_kv;                   // K/V heads; query head h reads K/V head h / (H / H_kv)
   int n_mtiles;               // ceil(N / 256)
+  int hgroup;                 // query heads per CTA-order group (>= 1; B*H: one group)
   float scale2;               // scale * log2(e)
   int causal;
 };
@@ -106,8 +107,15 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int BH = p.B * p.H;
-  const int mt = p.n_mtiles - 1 - static_cast<int>(blockIdx.x) / BH;  // heaviest tiles first
-  const int bh = static_cast<int>(blockIdx.x) % BH;
+  // CTA order: groups of p.hgroup heads in turn (a group's Q, K, V and O fit in L2), and
+  // inside a group the heaviest Q tiles (the last rows under a causal mask) first.
+  const int per_group = p.hgroup * p.n_mtiles;
+  const int grp = static_cast<int>(blockIdx.x) / per_group;
+  const int g0 = grp * p.hgroup;
+  const int gn = min(p.hgroup, BH - g0);               // heads in this group (the last may have fewer)
+  const int slot = static_cast<int>(blockIdx.x) - grp * per_group;
+  const int mt = p.n_mtiles - 1 - slot / gn;
+  const int bh = g0 + slot % gn;
   const int b = bh / p.H;
   const int bh_kv = b * p.H_kv + (bh % p.H) / (p.H / p.H_kv);  // K/V head of this query head
   const int N = p.N;
