@@ -77,6 +77,11 @@ def _load():
                                                 ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                                 ctypes.c_int, _u8p, ctypes.c_int, _i32p, _i64p,
                                                 ctypes.c_int, _dp]
+        lib.oracle_attn_bwd_kv_rows.restype = ctypes.c_int
+        lib.oracle_attn_bwd_kv_rows.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                                ctypes.c_int, _u8p, ctypes.c_int, _i32p, _i64p,
+                                                ctypes.c_int, _dp, _dp]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -177,6 +182,28 @@ def attn_bwd_dq_rows(q, k, v, do, scale: float, rows: Sequence[int], causal: boo
     if rc != 0:
         raise RuntimeError(f"oracle_attn_bwd_dq_rows failed ({rc})")
     return dq
+
+
+def attn_bwd_kv_rows(q, k, v, do, scale: float, rows: Sequence[int], causal: bool = False,
+                     block_mask=None, kv_len=None, block: int = 128):
+    """dK and dV of selected key rows (flat (b*H + h)*N + j), float64 [len(rows), d] each.
+    Every query row that may attend to a selected key is materialised in full (its softmax
+    normaliser and its sum over k are needed), so the cost is that of the full backward of
+    the heads that hold a selected key, without the N x N storage."""
+    lib = _load()
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, H, N, d = q.shape
+    bm, kl = _masks(block_mask, kv_len)
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    dk = np.zeros((len(r), d), np.float64)
+    dv = np.zeros((len(r), d), np.float64)
+    rc = lib.oracle_attn_bwd_kv_rows(_ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), _ptr(do, _dp),
+                                     B, H, N, d, float(scale), int(bool(causal)),
+                                     _ptr(bm, _u8p), block, _ptr(kl, _i32p), _ptr(r, _i64p),
+                                     len(r), _ptr(dk, _dp), _ptr(dv, _dp))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_bwd_kv_rows failed ({rc})")
+    return dk, dv
 
 
 def kv_group(H: int, H_kv: int) -> int:

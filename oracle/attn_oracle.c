@@ -354,3 +354,90 @@ int oracle_attn_bwd_dq_rows(const double *q, const double *k, const double *v, c
     }
     return bad ? -1 : 0;
 }
+
+/* dK and dV of selected key rows only (flat index (b*H + h)*N + j).  dK_j and dV_j are sums
+ * over the query rows i of column j of dS and of A:
+ *     dV_j = sum_i A_ij dO_i,    dK_j = scale * sum_i dS_ij q_i,
+ *     dS_ij = A_ij (dA_ij - sum_k A_ik dA_ik),   dA_ij = dO_i . v_j,
+ * and each A_ij, dS_ij needs the whole of row i (its normaliser and its sum over k).  So every
+ * row i that may attend to at least one selected key of its head is materialised in full (S,
+ * A and dA), exactly as in oracle_attn_bwd, and the entries of the selected columns are kept;
+ * the sums over i then run in index order.  Keys of heads with no selected key cost nothing. */
+int oracle_attn_bwd_kv_rows(const double *q, const double *k, const double *v, const double *dO,
+                            int B, int H, int N, int d, double scale, int causal,
+                            const uint8_t *block_mask, int block, const int32_t *kv_len,
+                            const int64_t *rows, int nrows, double *dk_rows, double *dv_rows)
+{
+    for (int r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] / N / H >= B) return -1;
+    /* column buffers: for selected key r, colA[r*N + i] = A_ij and colS[r*N + i] = dS_ij */
+    double *colA = (double *)calloc((size_t)nrows * (size_t)N, sizeof(double));
+    double *colS = (double *)calloc((size_t)nrows * (size_t)N, sizeof(double));
+    if ((!colA || !colS) && nrows > 0) { free(colA); free(colS); return -2; }
+    for (int bh = 0; bh < B * H; ++bh) {
+        /* the selected keys of this head */
+        int nsel = 0;
+        for (int r = 0; r < nrows; ++r) if (rows[r] / N == bh) ++nsel;
+        if (nsel == 0) continue;
+        int *sel = (int *)malloc(sizeof(int) * (size_t)nsel);
+        nsel = 0;
+        for (int r = 0; r < nrows; ++r) if (rows[r] / N == bh) sel[nsel++] = r;
+        int b = bh / H;
+        mask_t m = make_mask(N, causal, block_mask, block, kv_len, b);
+        size_t off = (size_t)bh * (size_t)N * d;
+        const double *qh = q + off, *kh = k + off, *vh = v + off, *dOh = dO + off;
+        #pragma omp parallel
+        {
+            double *a = (double *)malloc(sizeof(double) * (size_t)N);
+            double *da = (double *)malloc(sizeof(double) * (size_t)N);
+            #pragma omp for schedule(dynamic, 16)
+            for (int i = 0; i < N; ++i) {
+                int any = 0;
+                for (int s = 0; s < nsel; ++s)
+                    if (key_allowed(&m, i, (int)(rows[sel[s]] % N))) { any = 1; break; }
+                if (!any) continue;               /* A_ij = dS_ij = 0 for every selected j */
+                logits_row(qh + (size_t)i * d, kh, N, d, scale, &m, i, a);
+                softmax_row(a, N);
+                const double *dOi = dOh + (size_t)i * d;
+                double delta = 0.0;
+                for (int j = 0; j < N; ++j) {
+                    double dot = 0.0;
+                    const double *vj = vh + (size_t)j * d;
+                    for (int c = 0; c < d; ++c) dot += dOi[c] * vj[c];
+                    da[j] = dot;                   /* dA_ij */
+                    delta += a[j] * dot;
+                }
+                for (int s = 0; s < nsel; ++s) {
+                    int r = sel[s];
+                    int j = (int)(rows[r] % N);
+                    colA[(size_t)r * N + i] = a[j];
+                    colS[(size_t)r * N + i] = a[j] * (da[j] - delta);
+                }
+            }
+            free(a);
+            free(da);
+        }
+        #pragma omp parallel for schedule(static)
+        for (int s = 0; s < nsel; ++s) {
+            int r = sel[s];
+            double *gk = dk_rows + (size_t)r * d, *gv = dv_rows + (size_t)r * d;
+            for (int c = 0; c < d; ++c) { gk[c] = 0.0; gv[c] = 0.0; }
+            for (int i = 0; i < N; ++i) {
+                double ws = colS[(size_t)r * N + i], wa = colA[(size_t)r * N + i];
+                if (ws != 0.0) {
+                    const double *qi = qh + (size_t)i * d;
+                    for (int c = 0; c < d; ++c) gk[c] += ws * qi[c];
+                }
+                if (wa != 0.0) {
+                    const double *dOi = dOh + (size_t)i * d;
+                    for (int c = 0; c < d; ++c) gv[c] += wa * dOi[c];
+                }
+            }
+            for (int c = 0; c < d; ++c) gk[c] *= scale;
+        }
+        free(sel);
+    }
+    free(colA);
+    free(colS);
+    return 0;
+}

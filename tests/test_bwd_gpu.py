@@ -58,7 +58,7 @@ def test_bwd_small_elementwise(cuda_lib, case):
 WORKLOAD_HEADS = {
     "gpt2_causal": [0, 13, 50, 95],
     "bert_padding": [0, 17, 100, 255],
-    "block_sparse": [0, 31],
+    "block_sparse": [0, 3, 7, 12, 16, 21, 26, 31],   # both batch entries, 8 of 32 heads
     "long_causal": [0],
 }
 
@@ -112,3 +112,16 @@ def test_bwd_long_causal_all_heads(cuda_lib):
     assert np.abs(got - rq).max() / scale <= 2e-2
     assert np.abs(got - rq).mean() / scale <= 2e-3
     assert torch.isfinite(dq.float()).all()
+    # dK and dV of key rows in one head of every L2-sized group of heads (the CTAs run 4 heads at
+    # a time here), against the oracle's definition: edge keys of the first, middle and last KV
+    # tiles plus random keys
+    rng = np.random.default_rng(79)
+    keys = []
+    for h in (0, 5, 10, 15):
+        js = np.concatenate([[0, 1, 127, 128, N // 2, N - 129, N - 128, N - 1],
+                             rng.choice(N, 8, replace=False)])
+        keys.append(h * N + np.unique(js))
+    keys = np.concatenate(keys)
+    rk, rv = oracle.attn_bwd_kv_rows(x["q"], x["k"], x["v"], x["do"], x["scale"], keys, True)
+    compare_grad(f64(dk).reshape(-1, d)[keys], rk, "dK key rows")
+    compare_grad(f64(dv).reshape(-1, d)[keys], rv, "dV key rows")

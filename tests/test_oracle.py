@@ -309,3 +309,54 @@ def test_dq_rows_match_brute_force(case):
                                  None if L is None else np.array([L], np.int32), block)
     ref = np.array(gq)[rows]
     assert np.max(np.abs(dq - ref)) < 1e-12 * max(1.0, np.max(np.abs(ref)))
+
+
+@pytest.mark.parametrize("case", range(len(CASES)))
+def test_kv_rows_match_brute_force(case):
+    """dK and dV of selected key rows equal the brute-force chain rule on the same keys (every
+    mask kind, ragged lengths, keys listed out of order and one key twice)."""
+    N, d, causal, L, bml, block = CASES[case]
+    q, k, v, do = _case(N, d, causal, L, bml, block, 400 + case)
+    scale = 0.55
+    bm = None if bml is None else np.array(bml, np.uint8)
+    _, gk, gv = bf.backward_head(q.tolist(), k.tolist(), v.tolist(), do.tolist(), scale, causal,
+                                 bml, block, L)
+    rows = list(range(N))[::-1] + [N // 2]
+    dk, dv = oracle.attn_bwd_kv_rows(q[None, None], k[None, None], v[None, None],
+                                     do[None, None], scale, rows, causal, bm,
+                                     None if L is None else np.array([L], np.int32), block)
+    for got, ref in ((dk, np.array(gk)[rows]), (dv, np.array(gv)[rows])):
+        assert np.max(np.abs(got - ref)) < 1e-12 * max(1.0, np.max(np.abs(ref)))
+
+
+def test_kv_rows_match_full_backward_across_heads():
+    """Across batch entries and heads (per-batch key lengths, a block mask with a fully masked
+    query block), the key-row entry reproduces the full backward's dK and dV rows, and keys
+    beyond a batch entry's length get exactly 0."""
+    B, H, N, d = 2, 3, 48, 6
+    q, k, v, do = (rand(B, H, N, d) for _ in range(4))
+    L = np.array([37, 48], np.int32)
+    bm = np.ones((3, 3), np.uint8)
+    bm[1, :] = 0            # query rows 16..31 see no key
+    bm[2, 0] = 0
+    for causal in (False, True):
+        _, dk, dv = oracle.attn_bwd(q, k, v, do, 0.4, causal, bm, L, block=16)
+        rng = np.random.default_rng(5)
+        rows = np.concatenate([rng.choice(B * H * N, 40, replace=False), [0, N - 1, B * H * N - 1]])
+        gk, gv = oracle.attn_bwd_kv_rows(q, k, v, do, 0.4, rows, causal, bm, L, block=16)
+        ref_k, ref_v = dk.reshape(-1, d)[rows], dv.reshape(-1, d)[rows]
+        assert np.max(np.abs(gk - ref_k)) < 1e-13 * max(1.0, np.abs(ref_k).max())
+        assert np.max(np.abs(gv - ref_v)) < 1e-13 * max(1.0, np.abs(ref_v).max())
+        pad = [r for r in range(N) if r >= 37]       # batch 0, head 0, padded keys
+        zk, zv = oracle.attn_bwd_kv_rows(q, k, v, do, 0.4, pad, causal, bm, L, block=16)
+        assert np.all(zk == 0.0) and np.all(zv == 0.0)
+
+
+def test_kv_rows_sum_invariants():
+    """Summed over every key of a head, dK is 0 and dV is the sum of dO over rows with a key --
+    the backward invariants, now through the key-row entry."""
+    N, d = 30, 4
+    q, k, v, do = (rand(1, 1, N, d) for _ in range(4))
+    dk, dv = oracle.attn_bwd_kv_rows(q, k, v, do, 0.7, list(range(N)), True)
+    assert np.max(np.abs(dk.sum(axis=0))) < 1e-12
+    assert np.max(np.abs(dv.sum(axis=0) - do[0, 0].sum(axis=0))) < 1e-12
