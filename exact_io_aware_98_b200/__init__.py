@@ -42,6 +42,10 @@ SIGNATURES = {
                           _vp]),
     "fa_diag_exp2": (_i, [_vp, _vp, _vp, _vp, _i, _vp]),
     "fa_diag_wait_timeout": (_i, [_i, _vp]),
+    "fa_launch_count": (ctypes.c_ulonglong, []),
+    "fa_kernel_timing": (_i, [_i]),
+    "fa_kernel_timing_read": (_i, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_int),
+                                   ctypes.POINTER(ctypes.c_double)]),
     "fa_get_last_error": (ctypes.c_char_p, []),
     "fa_device_status": (_i, [ctypes.POINTER(ctypes.c_uint)]),
 }
@@ -155,6 +159,31 @@ def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
     return int(load().fa_bwd_workspace_size(B, H, N, d))
 
 
+def _bwd_operands(q, k, v, o, lse, do, dq, dk, dv):
+    """Checks shared by every backward call: dtypes, contiguity, and the shapes of o, do, lse
+    and of caller-supplied gradients against q, k and v (so that no kernel is ever handed a
+    buffer smaller than the tensor maps it builds from q's sizes).  Returns H_kv and dq, dk, dv
+    (allocated here when not supplied)."""
+    B, H, N, d = q.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _require(t, n, q.dtype)
+    H_kv = _kv_heads(q, k, v)
+    for t, n in ((o, "o"), (do, "do")):
+        if t.shape != q.shape:
+            raise FaError(f"{n} shape {tuple(t.shape)} does not match q {tuple(q.shape)}")
+    _require(lse, "lse", torch.float32)
+    if tuple(lse.shape) != (B, H, N):
+        raise FaError(f"lse shape {tuple(lse.shape)} must be {(B, H, N)}")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _require(t, n, q.dtype)
+    if dq.shape != q.shape or dk.shape != k.shape or dv.shape != v.shape:
+        raise FaError("gradient shapes must match q, k and v")
+    return H_kv, dq, dk, dv
+
+
 def bwd(q, k, v, o, lse, do, scale: Optional[float] = None, causal: bool = False,
         block_mask=None, kv_len=None, workspace=None, dq=None, dk=None, dv=None,
         deterministic: bool = False):
@@ -163,20 +192,10 @@ def bwd(q, k, v, o, lse, do, scale: Optional[float] = None, causal: bool = False
     bit-reproducible gradients, dQ without atomics."""
     lib = load()
     B, H, N, d = q.shape
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
-        _require(t, n, q.dtype)
-    H_kv = _kv_heads(q, k, v)
-    _require(lse, "lse", torch.float32)
+    H_kv, dq, dk, dv = _bwd_operands(q, k, v, o, lse, do, dq, dk, dv)
     need = bwd_workspace_size(B, H, N, d)
     ws = torch.empty(need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
     _require(ws, "workspace", torch.uint8)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
-    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
-        _require(t, n, q.dtype)
-    if dq.shape != q.shape or dk.shape != k.shape or dv.shape != v.shape:
-        raise FaError("gradient shapes must match q, k and v")
     bm, kl = _masks(block_mask, kv_len)
     s = default_scale(d) if scale is None else float(scale)
     if deterministic:
@@ -200,16 +219,17 @@ def bwd(q, k, v, o, lse, do, scale: Optional[float] = None, causal: bool = False
 
 def bwd_noalloc(q, k, v, o, lse, do, scale: Optional[float] = None, causal: bool = False,
                 block_mask=None, kv_len=None, dq=None, dk=None, dv=None):
-    """fa_bwd without a workspace: for callers that cannot allocate device memory.  The
-    library's own fixed 32 MiB scratch is used instead; calls on one device must not overlap."""
+    """fa_bwd without a workspace, for callers that cannot allocate device memory: the
+    library's own fixed 32 MiB scratch is used instead, and calls on one device must not
+    overlap.  Ordinary attention only (k and v have q's H heads).  dq, dk and dv may be passed
+    in; otherwise this wrapper allocates them with torch, which a caller that cannot allocate
+    avoids by passing its own."""
     lib = load()
     B, H, N, d = q.shape
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
-        _require(t, n, q.dtype)
-    _require(lse, "lse", torch.float32)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
+    H_kv, dq, dk, dv = _bwd_operands(q, k, v, o, lse, do, dq, dk, dv)
+    if H_kv != H:
+        raise FaError(f"fa_bwd_noalloc takes ordinary attention only (k/v have {H_kv} heads, "
+                      f"q has {H})")
     bm, kl = _masks(block_mask, kv_len)
     s = default_scale(d) if scale is None else float(scale)
     rc = lib.fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq),
@@ -285,3 +305,23 @@ def device_status() -> int:
     if rc not in (0, -5):
         _check(rc, "fa_device_status")
     return int(code.value)
+
+
+def launch_count() -> int:
+    """Kernels this library has launched in the process (fa_launch_count)."""
+    return int(load().fa_launch_count())
+
+
+def kernel_timing(enable: bool):
+    """Start (True) or stop (False) bracketing each tensor-core launch with CUDA events."""
+    _check(load().fa_kernel_timing(int(bool(enable))), "fa_kernel_timing")
+
+
+def kernel_timing_read(name: str = ""):
+    """(launches, total ms) of the recorded launches of kernels whose name contains ``name``;
+    waits for them and forgets them."""
+    n = ctypes.c_int(0)
+    ms = ctypes.c_double(0.0)
+    _check(load().fa_kernel_timing_read(name.encode(), ctypes.byref(n), ctypes.byref(ms)),
+           "fa_kernel_timing_read")
+    return int(n.value), float(ms.value)

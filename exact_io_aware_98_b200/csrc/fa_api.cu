@@ -4,11 +4,13 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "fa.h"
 #include "fa_bwd_dkdv_sm100.cuh"
@@ -32,11 +34,58 @@ int fail(int code, const char* fmt, ...) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+std::atomic<unsigned long long> g_launches{0};
+
 int check_launch(const char* what) {
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(FA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   return FA_OK;
 }
+
+// ---- optional per-kernel timing (fa_kernel_timing): two events around each tensor-core launch
+struct TimingRecord {
+  const char* kernel;
+  cudaEvent_t start, stop;
+};
+std::mutex g_timing_mu;
+std::atomic<bool> g_timing_on{false};
+std::vector<TimingRecord> g_timing;      // recorded, not yet read
+std::vector<cudaEvent_t> g_event_pool;   // created once, reused
+
+cudaEvent_t pooled_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Brackets one launch with events on its stream while timing is enabled; otherwise inert.
+class TimedLaunch {
+ public:
+  TimedLaunch(const char* kernel, cudaStream_t s) : kernel_(kernel), s_(s) {
+    if (!g_timing_on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lock(g_timing_mu);
+    start_ = pooled_event();
+    stop_ = pooled_event();
+    if (start_ != nullptr && stop_ != nullptr) cudaEventRecord(start_, s_);
+  }
+  ~TimedLaunch() {
+    if (start_ == nullptr || stop_ == nullptr) return;
+    cudaEventRecord(stop_, s_);
+    std::lock_guard<std::mutex> lock(g_timing_mu);
+    g_timing.push_back({kernel_, start_, stop_});
+  }
+
+ private:
+  const char* kernel_;
+  cudaStream_t s_;
+  cudaEvent_t start_ = nullptr, stop_ = nullptr;
+};
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -162,6 +211,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.causal = causal ? 1 : 0;
   const long long grid = static_cast<long long>(p.n_mtiles) * BH;
   if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
+  TimedLaunch tl("fa_fwd_sm100_kernel", stream);
   fa::fa_fwd_sm100_kernel<D><<<static_cast<unsigned>(grid), 320, L::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
   return check_launch("fa_fwd_sm100_kernel");
 }
@@ -210,6 +260,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void
   }
   const long long grid = static_cast<long long>(p.n_ktiles) * B * H_kv;  // one CTA per K/V tile
   if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
+  TimedLaunch tl("fa_bwd_sm100_kernel", stream);
   fa::fa_bwd_sm100_kernel<D><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, mdq, p);
   return check_launch("fa_bwd_sm100_kernel");
 }
@@ -249,6 +300,7 @@ int launch_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
   p.causal = causal ? 1 : 0;
   const long long grid = static_cast<long long>(p.n_ktiles) * B * H_kv;
   if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
+  TimedLaunch tl("fa_bwd_dkdv_sm100_kernel", stream);
   fa::fa_bwd_dkdv_sm100_kernel<D><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
   return check_launch("fa_bwd_dkdv_sm100_kernel");
 }
@@ -284,6 +336,7 @@ int launch_bwd_dq(const void* q, const void* k, const void* v, const void* dO, v
   p.causal = causal ? 1 : 0;
   const long long grid = static_cast<long long>(p.n_mtiles) * BH;
   if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
+  TimedLaunch tl("fa_bwd_dq_sm100_kernel", stream);
   fa::fa_bwd_dq_sm100_kernel<D><<<static_cast<unsigned>(grid), 320, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
   return check_launch("fa_bwd_dq_sm100_kernel");
 }
@@ -498,6 +551,48 @@ int fa_diag_exp2(const float* x, float* y_fma, float* y_mufu, float* y_ref, int 
   return check_launch("diag_exp2_kernel");
 }
 
+unsigned long long fa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int fa_kernel_timing(int enable) {
+  g_timing_on.store(enable != 0, std::memory_order_relaxed);
+  return FA_OK;
+}
+
+int fa_kernel_timing_read(const char* name, int* launches, double* total_ms) {
+  if (name == nullptr || launches == nullptr || total_ms == nullptr)
+    return fail(FA_ERR_INVALID, "null pointer");
+  std::vector<TimingRecord> mine;
+  {
+    std::lock_guard<std::mutex> lock(g_timing_mu);
+    std::vector<TimingRecord> rest;
+    for (const TimingRecord& r : g_timing)
+      (std::strstr(r.kernel, name) != nullptr ? mine : rest).push_back(r);
+    g_timing.swap(rest);
+  }
+  int n = 0;
+  double ms = 0.0;
+  int rc = FA_OK;
+  for (const TimingRecord& r : mine) {
+    float t = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.stop);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.start, r.stop);
+    if (e != cudaSuccess && rc == FA_OK)
+      rc = fail(FA_ERR_CUDA, "kernel timing: %s", cudaGetErrorString(e));
+    ++n;
+    ms += t;
+  }
+  {
+    std::lock_guard<std::mutex> lock(g_timing_mu);
+    for (const TimingRecord& r : mine) {
+      g_event_pool.push_back(r.start);
+      g_event_pool.push_back(r.stop);
+    }
+  }
+  *launches = n;
+  *total_ms = ms;
+  return rc;
+}
+
 int fa_diag_wait_timeout(int site, void* stream) {
   if (site < 1 || site > 0x7fff) return fail(FA_ERR_INVALID, "site must be in [1, 32767]");
   fa::diag_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(site);
@@ -557,25 +652,62 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
+struct NoallocSlot {
+  void* ptr = nullptr;           // device address of g_noalloc_scratch in context `ctx_id`
+  unsigned long long ctx_id = 0;
+  bool have_id = false;
+};
+NoallocSlot g_noalloc[kMaxDevices];
 
-// Device address of g_noalloc_scratch on the current device.  The host-side name of the array
-// is only a stand-in, never a device address, so the address is looked up once per device (with
-// that device current) and cached.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult qres;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &qres) != cudaSuccess ||
+      qres != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
+
+// Unique id of the CUDA context current on this thread (a context made after cudaDeviceReset
+// gets a new id even if it lands at the same handle value); false if there is none or the
+// driver cannot say.
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_cur = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (get_cur == nullptr || get_id == nullptr) return false;
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_noalloc_scratch in the current context.  The host-side name of the array
+// is only a stand-in, never a device address, so the address is looked up with the device
+// current.  It is cached per device together with the id of the context it was looked up in,
+// and looked up again whenever another context is current (after cudaDeviceReset, or with a
+// context the caller made): the module -- and the array with it -- is loaded anew per context.
 int noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return fail(FA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id);
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  NoallocSlot& slot = g_noalloc[dev];
+  if (slot.ptr == nullptr || !have_id || !slot.have_id || slot.ctx_id != id) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr)
       return fail(FA_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
-    g_noalloc_ptr[dev] = p;
+    slot.ptr = p;
+    // the lookup made the device's context current if none was: record the id it has now
+    slot.have_id = current_context_id(&slot.ctx_id);
   }
-  *out = g_noalloc_ptr[dev];
+  *out = slot.ptr;
   return FA_OK;
 }
 

@@ -102,8 +102,11 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
  *   Arguments, layouts, masks and results are those of fa_bwd, without the workspace pair.
  *   Limit: problems whose fa_bwd_workspace_size(B, H, N, d) exceeds 32 MiB (33554432 bytes)
  *   are rejected with FA_ERR_WORKSPACE before anything is launched.
- *   Set-up: the first call on a device looks up the array's device address (with that device
- *   current) and caches it; make that first call before any stream capture.
+ *   Set-up: the array's device address is looked up with the device current and cached
+ *   together with the id of the CUDA context it belongs to.  The first call on a device, and
+ *   the first call after the current context changes (cudaDeviceReset, or a context the caller
+ *   made current), does that look-up; later calls only compare the context id.  Make the first
+ *   call in each context before any stream capture.
  *   Sharing: every call on a device uses the same scratch and leaves its contents behind; each
  *   call re-initialises everything it reads, but two calls that overlap on the GPU (different
  *   streams, no ordering between them) race on the scratch and give wrong gradients.
@@ -199,6 +202,26 @@ int fa_diag_exp2(const float* x, float* y_fma, float* y_mufu, float* y_ref, int 
  * fa_device_status() then reports FA_ERR_TIMEOUT with code (site << 16).  Nothing traps.
  */
 int fa_diag_wait_timeout(int site, void* stream);
+
+/*
+ * Measurement diagnostics (no counterpart on the pages; they let a benchmark count and time this
+ * library's own kernels from inside a timed region).
+ *   fa_launch_count       -- number of kernels this library has launched in the process, over
+ *                            every entry point and device (a launch the driver rejected is not
+ *                            counted).
+ *   fa_kernel_timing      -- enable != 0: from now on every launch of a tensor-core kernel
+ *                            (fa_fwd_sm100_kernel, fa_bwd_sm100_kernel, fa_bwd_dkdv_sm100_kernel,
+ *                            fa_bwd_dq_sm100_kernel) is bracketed by two CUDA events recorded on
+ *                            the launch's stream; enable == 0 stops recording.  Off by default.
+ *   fa_kernel_timing_read -- waits for the recorded launches of every kernel whose name contains
+ *                            `name` ("" = all), stores how many there were in *launches and the
+ *                            sum of their event-measured durations in *total_ms, and forgets
+ *                            them.  FA_ERR_INVALID for a null pointer; FA_ERR_CUDA if an event
+ *                            query fails (the counts are still stored).
+ */
+unsigned long long fa_launch_count(void);
+int fa_kernel_timing(int enable);
+int fa_kernel_timing_read(const char* name, int* launches, double* total_ms);
 
 /* Message for the most recent non-OK status returned on this host thread. */
 const char* fa_get_last_error(void);

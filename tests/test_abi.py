@@ -143,3 +143,15 @@ def test_binding_raises_when_library_missing(tmp_path):
             fa.load(str(tmp_path / "nope.so"))
     finally:
         fa._lib = saved
+
+
+def test_measurement_diagnostics_without_a_gpu(lib):
+    """The launch counter and the kernel-timing switch work on the host: no launch has been
+    made in this process, so nothing is counted or recorded; a null output is rejected."""
+    assert lib.fa_launch_count() == 0
+    assert lib.fa_kernel_timing(1) == OK
+    n, ms = ctypes.c_int(-1), ctypes.c_double(-1.0)
+    assert lib.fa_kernel_timing_read(b"", ctypes.byref(n), ctypes.byref(ms)) == OK
+    assert n.value == 0 and ms.value == 0.0
+    assert lib.fa_kernel_timing(0) == OK
+    assert lib.fa_kernel_timing_read(b"fa_", None, ctypes.byref(ms)) == INVALID
