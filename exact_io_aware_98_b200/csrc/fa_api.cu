@@ -190,8 +190,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   const int BH = B * H;
   int rc;
   if ((rc = make_map(&mq, q, BH, N, D, 128, "q")) != FA_OK) return rc;
-  if ((rc = make_map(&mk, k, B * H_kv, N, D, 128, "k")) != FA_OK) return rc;
-  if ((rc = make_map(&mv, v, B * H_kv, N, D, 128, "v")) != FA_OK) return rc;
+  if ((rc = make_map(&mk, k, B * H_kv, N, D, L::BN, "k")) != FA_OK) return rc;
+  if ((rc = make_map(&mv, v, B * H_kv, N, D, L::BN, "v")) != FA_OK) return rc;
   if ((rc = set_smem(fa::fa_fwd_sm100_kernel<D>, L::SMEM_ALLOC)) != FA_OK) return rc;
   fa::FwdParams p;
   p.block_mask = bm;

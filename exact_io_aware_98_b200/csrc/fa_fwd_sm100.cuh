@@ -9,17 +9,23 @@
 // running normalisation; accumulate the output without materialising the full matrix;
 // schedule for the target accelerator).
 //
-// CTA layout (320 threads, one CTA per SM):
+// CTA layout (320 threads):
 //   warps 0-3  softmax warpgroup for Q tile 0 (rows m0 .. m0+127), one thread per row
 //   warps 4-7  softmax warpgroup for Q tile 1 (rows m0+128 .. m0+255)
-//   warp  8    TMA producer: Q once, then K and V tiles of 128 keys through separate rings
+//   warp  8    TMA producer: Q once, then K and V tiles of BN keys through separate rings
 //              (a K stage frees as soon as both S MMAs of its tile finish, a V stage after
 //              both PV MMAs, so K runs further ahead than a shared ring would allow)
 //   warp  9    MMA issuer (whole warp, one elected lane issues): S_w = Q_w K^T into TMEM,
 //              O_w += P_w V with P taken from TMEM
-// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [256+D,256+2D).
-// P_w (bf16, two per 32-bit column) overwrites columns [0,64) of S_w after the softmax
-// warpgroup has read S_w into registers.
+// TMEM: S_0 [0,BN), S_1 [BN,2BN), O_0 [2BN,2BN+D), O_1 [2BN+D,2BN+2D).  P_w (bf16, two per
+// 32-bit column) overwrites columns [0,BN/2) of S_w after the softmax warpgroup has read S_w
+// into registers.
+// Key-tile width BN: 128 at d = 128 (one CTA per SM, all 512 TMEM columns).  At d = 64 it is
+// 64, which halves TMEM (256 columns) and shared memory (~100 KB) per CTA so that two CTAs share
+// an SM: the head dimension is small, the softmax (one exponential per score whatever d is)
+// dominates, and one CTA's set-up, first loads and epilogue -- about 5 us between consecutive
+// CTAs on an SM, measured -- then overlap the other CTA's loop, while four softmax warpgroups
+// per SM keep the exponential units busy during each other's MMA round trips.
 //
 // Per KV tile the MMA thread issues, for w = 0 then 1: PV_w of the previous tile, then S_w of
 // this tile.  tcgen05 MMAs from one thread execute in issue order, so S_w(t+1) cannot overwrite
@@ -53,26 +59,31 @@ struct FwdParams {
 template <int D>
 struct FwdLayout {
   static constexpr int BM = 128;                    // query rows per Q tile
-  static constexpr int BN = 128;                    // keys per KV tile
-  static constexpr int KST = D == 64 ? 5 : 3;       // K ring depth
+  static constexpr int BN = D == 64 ? 64 : 128;     // keys per KV tile
+  static constexpr int CTAS_PER_SM = D == 64 ? 2 : 1;
+  static constexpr int KST = D == 64 ? 4 : 3;       // K ring depth
   static constexpr int VST = D == 64 ? 4 : 2;       // V ring depth
   static constexpr int SUB = D / 64;                // 64-column (128-byte) sub-tiles
-  static constexpr int SUBTILE = 128 * 128;         // bytes of one 128-row x 64-col sub-tile
-  static constexpr int TILE = 128 * D * 2;          // bytes of one 128-row tile
+  static constexpr int SUBTILE = 128 * 128;         // bytes of one 128-row x 64-col Q sub-tile
+  static constexpr int TILE = 128 * D * 2;          // bytes of one 128-row Q tile
+  static constexpr int KV_SUBTILE = BN * 128;       // bytes of one BN-row x 64-col K/V sub-tile
+  static constexpr int KV_TILE = BN * D * 2;        // bytes of one K or V tile
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * TILE;
-  static constexpr int OFF_V = OFF_K + KST * TILE;
-  static constexpr int OFF_BAR = OFF_V + VST * TILE;
+  static constexpr int OFF_V = OFF_K + KST * KV_TILE;
+  static constexpr int OFF_BAR = OFF_V + VST * KV_TILE;
   // q, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], p_full[2], o_done[2], fin
   static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 6 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;   // slack for 1024-byte alignment
-  static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t O_COL0 = 256;
+  static_assert(CTAS_PER_SM * (SMEM_ALLOC + 1024) <= 233472, "shared memory per SM");
+  static constexpr uint32_t TMEM_COLS = D == 64 ? 256 : 512;
+  static constexpr uint32_t O_COL0 = 2 * BN;
+  static_assert(O_COL0 + 2 * D <= TMEM_COLS, "TMEM budget");
   // one P pair in EMU_EVERY is exponentiated on the FMA pipe (0 = all on MUFU)
   static constexpr int EMU_EVERY = 4;
-  __device__ static constexpr uint32_t s_col(int w) { return static_cast<uint32_t>(w) * 128u; }
+  __device__ static constexpr uint32_t s_col(int w) { return static_cast<uint32_t>(w) * BN; }
 };
 
 // Wait-site codes recorded in the status word on a timeout.
@@ -83,7 +94,7 @@ enum : int {
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(320, FwdLayout<D>::CTAS_PER_SM)
 fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -122,22 +133,24 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int m0 = mt * 256;
   int kvlen = N;
   if (p.kv_len != nullptr) kvlen = min(max(p.kv_len[b], 0), N);
-  const int nb = (N + 127) / 128;
-  const int n_kv = (kvlen + 127) / 128;
+  constexpr int BN = L::BN;
+  const int nb = (N + 127) / 128;                      // 128 x 128 blocks of the block mask
+  const int n_kv = (kvlen + BN - 1) / BN;
   int j_end = n_kv;
-  if (p.causal) j_end = min(j_end, (min(m0 + 256, N) - 1) / 128 + 1);
+  if (p.causal) j_end = min(j_end, (min(m0 + 256, N) - 1) / BN + 1);
 
   // bit w set: KV tile j holds at least one key that Q tile w may attend to
   auto flags_of = [&](int j) -> int {
     int f = 0;
-    const int k0 = j * 128;
+    const int k0 = j * BN;
 #pragma unroll
     for (int w = 0; w < 2; ++w) {
       const int q0 = m0 + 128 * w;
       if (q0 >= N) continue;
       const int q1 = min(q0 + 127, N - 1);
       if (p.causal && k0 > q1) continue;
-      if (p.block_mask != nullptr && !p.block_mask[static_cast<size_t>(q0 >> 7) * nb + j]) continue;
+      if (p.block_mask != nullptr && !p.block_mask[static_cast<size_t>(q0 >> 7) * nb + (k0 >> 7)])
+        continue;
       f |= 1 << w;
     }
     return f;
@@ -190,18 +203,18 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (kn >= L::KST &&
             !mbar_wait(&bar_ke[ks], ((kn / L::KST) - 1) & 1, abort_flag, SITE_FWD_LOAD_EMPTY))
           break;
-        mbar_arrive_expect_tx(&bar_kf[ks], L::TILE);
+        mbar_arrive_expect_tx(&bar_kf[ks], L::KV_TILE);
         for (int s = 0; s < L::SUB; ++s)
-          tma_load_3d(smem + L::OFF_K + ks * L::TILE + s * L::SUBTILE, &tm_k, &bar_kf[ks], s * 64,
-                      j * 128, bh_kv);
+          tma_load_3d(smem + L::OFF_K + ks * L::KV_TILE + s * L::KV_SUBTILE, &tm_k, &bar_kf[ks],
+                      s * 64, j * BN, bh_kv);
         ++kn;
         if (vn >= L::VST &&
             !mbar_wait(&bar_ve[vs], ((vn / L::VST) - 1) & 1, abort_flag, SITE_FWD_LOAD_EMPTY))
           break;
-        mbar_arrive_expect_tx(&bar_vf[vs], L::TILE);
+        mbar_arrive_expect_tx(&bar_vf[vs], L::KV_TILE);
         for (int s = 0; s < L::SUB; ++s)
-          tma_load_3d(smem + L::OFF_V + vs * L::TILE + s * L::SUBTILE, &tm_v, &bar_vf[vs], s * 64,
-                      j * 128, bh_kv);
+          tma_load_3d(smem + L::OFF_V + vs * L::KV_TILE + s * L::KV_SUBTILE, &tm_v, &bar_vf[vs],
+                      s * 64, j * BN, bh_kv);
         ++vn;
       }
       // Never leave the CTA with a copy in flight: wait for the last loads of every stage
@@ -215,16 +228,18 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
     // The whole warp walks the loop (descriptors stay warp-uniform); one elected lane issues.
-    constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, BN, false, false);
     constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
     // Base descriptors; stage, sub-tile and K-step offsets are added to the start-address
     // field (16-byte units).  Q/K: K-major, 128-byte rows, 8-row groups 1 KB apart.
     // V: MN-major, 64-column blocks one sub-tile apart.
     const uint64_t q_desc = sdesc_sw128(smem_u32(smem + L::OFF_Q), 16, 1024);
     const uint64_t k_desc = sdesc_sw128(smem_u32(smem + L::OFF_K), 16, 1024);
-    const uint64_t v_desc = sdesc_sw128(smem_u32(smem + L::OFF_V), L::SUBTILE, 1024);
-    auto koff = [](int k) -> uint64_t {  // K-step k of a K-major operand, in 16-byte units
-      return static_cast<uint64_t>(((k >> 2) * L::SUBTILE + (k & 3) * 32) >> 4);
+    const uint64_t v_desc = sdesc_sw128(smem_u32(smem + L::OFF_V), L::KV_SUBTILE, 1024);
+    // K-step k of a K-major operand whose 64-column sub-tiles are `sub` bytes apart, in
+    // 16-byte units
+    auto koff = [](int k, int sub) -> uint64_t {
+      return static_cast<uint64_t>(((k >> 2) * sub + (k & 3) * 32) >> 4);
     };
     bool ok = mbar_wait_w(bar_q, 0, abort_flag, SITE_FWD_MMA_Q);
     tc_fence_after();
@@ -237,7 +252,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       tc_fence_after();
       const uint32_t a_tmem = tmem + L::s_col(w);
       const uint32_t d_tmem = tmem + L::O_COL0 + w * D;
-      const uint64_t vb = v_desc + static_cast<uint64_t>((vs * L::TILE) >> 4);
+      const uint64_t vb = v_desc + static_cast<uint64_t>((vs * L::KV_TILE) >> 4);
 #pragma unroll
       for (int kb = 0; kb < L::BN / 64; ++kb) {
         uint32_t a[4];
@@ -257,14 +272,14 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     // S_w = Q_w K(ks)^T
     auto issue_s = [&](int w, int ks) {
       const uint64_t qa = q_desc + static_cast<uint64_t>((w * L::TILE) >> 4);
-      const uint64_t kb0 = k_desc + static_cast<uint64_t>((ks * L::TILE) >> 4);
+      const uint64_t kb0 = k_desc + static_cast<uint64_t>((ks * L::KV_TILE) >> 4);
 #pragma unroll
       for (int kb = 0; kb < D / 64; ++kb) {
         uint64_t a[4], b[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          a[i] = qa + koff(4 * kb + i);
-          b[i] = kb0 + koff(4 * kb + i);
+          a[i] = qa + koff(4 * kb + i, L::SUBTILE);
+          b[i] = kb0 + koff(4 * kb + i, L::KV_SUBTILE);
         }
         mma_ss_x4(tmem + L::s_col(w), a, b, idesc_s, kb > 0 ? 1u : 0u);
       }
@@ -324,17 +339,18 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const bool got = mbar_wait(&bar_sf[w], cnt & 1, abort_flag, SITE_FWD_SM_S);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
-      uint32_t r[4][32];
+      constexpr int NC = BN / 32;  // 32-column chunks of S_w
+      uint32_t r[NC][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(t_s + 32 * c, r[c]);
+      for (int c = 0; c < NC; ++c) tmem_ld32(t_s + 32 * c, r[c]);
       tmem_ld_wait();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence(r[c]);
-      const int k0 = j * 128;
-      const bool edge = (k0 + 128 > kvlen) || (p.causal && k0 + 127 > q0 + 32 * qw);
+      for (int c = 0; c < NC; ++c) reg_fence(r[c]);
+      const int k0 = j * BN;
+      const bool edge = (k0 + BN > kvlen) || (p.causal && k0 + BN - 1 > q0 + 32 * qw);
       if (edge) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < NC; ++c)
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int col = k0 + 32 * c + i;
@@ -346,7 +362,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
       for (int u = 0; u < 8; ++u) mc[u] = -INFINITY;
 #pragma unroll
-      for (int k = 0; k < 128; k += 2)
+      for (int k = 0; k < BN; k += 2)
         mc[(k >> 1) & 7] = fmax3(mc[(k >> 1) & 7], __uint_as_float(r[k >> 5][k & 31]),
                                  __uint_as_float(r[k >> 5][(k & 31) + 1]));
       const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]),
@@ -360,10 +376,10 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       // independent accumulator pairs).  On tiles without masked elements, one pair in
       // L::EMU_EVERY takes 2^x on the FMA pipe instead of MUFU, which the other pairs keep busy.
       float ra[4] = {0.f, 0.f, 0.f, 0.f}, rb[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[4][16];
+      uint32_t pk[NC][16];
       auto exp_pairs = [&](bool use_fma) {
 #pragma unroll
-        for (int q = 0; q < 64; ++q) {
+        for (int q = 0; q < BN / 2; ++q) {
           const int c = q >> 4, i = q & 15;
           float x0, x1, p0, p1;
           ffma2(x0, x1, __uint_as_float(r[c][2 * i]), __uint_as_float(r[c][2 * i + 1]), scale2,
@@ -382,7 +398,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       else exp_pairs(true);
       l = alpha * l + ((ra[0] + ra[1]) + (ra[2] + ra[3]) + ((rb[0] + rb[1]) + (rb[2] + rb[3])));
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_st16(t_s + 16 * c, pk[c]);
+      for (int c = 0; c < NC; ++c) tmem_st16(t_s + 16 * c, pk[c]);
       const bool rescale = (cnt > 0) && (m_new != m_ref);
       if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll

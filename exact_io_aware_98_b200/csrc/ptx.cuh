@@ -73,6 +73,50 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// The same bounded wait without the abort flag, for draining an asynchronous operation that
+// is already in flight (its completion must be seen before the CTA may exit).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 15u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicCAS(&g_status, 0u, (static_cast<unsigned>(site) << 16) | (blockIdx.x & 0xffffu));
+      return false;
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------- work stealing
+// Cluster launch control (sm_100): ask the hardware to cancel the launch of a CTA of this grid
+// that has not started yet; on success its work falls to the asking CTA.  The 16-byte response
+// is written to `resp16` (shared, 16-byte aligned) by the async proxy and completes 16 bytes of
+// transactions on `bar` (arm it with mbar_arrive_expect_tx(bar, 16) first).  Only one request
+// may be in flight per response buffer, and none may follow a failed one.
+__device__ __forceinline__ void clc_try_cancel(void* resp16, uint64_t* bar) {
+  asm volatile(
+      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128"
+      " [%0], [%1];" ::"r"(smem_u32(resp16)),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+// Reads a completed response: the x index of the cancelled CTA, or -1 if none was cancelled.
+// Ends with a proxy fence, so the buffer may take the next request's response afterwards.
+__device__ __forceinline__ int clc_cancelled_x(const void* resp16) {
+  uint32_t x = 0, ok = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b128 c;\n\t"
+      "ld.shared.b128 c, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, c;\n\t"
+      "selp.u32 %1, 1, 0, p;\n\t"
+      "@p clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %0, c;\n\t}\n"
+      : "=r"(x), "=r"(ok)
+      : "r"(smem_u32(resp16))
+      : "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  return ok ? static_cast<int>(x) : -1;
+}
+
 // ----------------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1, int c2) {
