@@ -286,7 +286,13 @@ int launch_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
   p.lse2 = reinterpret_cast<const float*>(wsb + ws.lse2);
   p.dvec = reinterpret_cast<const float*>(wsb + ws.dvec);
   p.dq_acc = nullptr;
-  p.hgroup = B * H_kv;                                   // not read by the dK/dV kernel
+  {
+    // K/V heads per CTA-order group: the group's Q and dO, 4 bytes per element of its G query
+    // heads, within half of the 126 MB L2.
+    const long long per_head = 4ll * (H / H_kv) * N * D;
+    p.hgroup = static_cast<int>(
+        std::max(1ll, std::min((64ll << 20) / per_head, static_cast<long long>(B) * H_kv)));
+  }
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.B = B;
@@ -331,6 +337,10 @@ int launch_bwd_dq(const void* q, const void* k, const void* v, const void* dO, v
   p.N = N;
   p.N_pad = ws.n_pad;
   p.n_mtiles = (N + 127) / 128;
+  // Query heads per CTA-order group: the K and V they read (4 bytes per element, counted per
+  // query head) within half of the 126 MB L2.
+  p.hgroup = static_cast<int>(
+      std::max(1ll, std::min((64ll << 20) / (4ll * N * D), static_cast<long long>(BH))));
   p.scale = scale;
   p.scale2 = scale * kLog2e;
   p.causal = causal ? 1 : 0;
@@ -447,12 +457,17 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
         block_mask, kv_len, B, H, H_kv, N, d, scale, causal ? 1 : 0);
     return check_launch("fa_bwd_f32_dkdv_kernel");
   }
-  const long long pre_rows = static_cast<long long>(BH) * ws.n_pad;
-  fa::bwd_preprocess_kernel<<<static_cast<unsigned>((pre_rows + 7) / 8), 256, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse,
-      reinterpret_cast<float*>(wsb + ws.lse2), reinterpret_cast<float*>(wsb + ws.dvec),
-      deterministic ? nullptr : reinterpret_cast<float*>(wsb + ws.dq), BH, N, ws.n_pad, d);
-  if ((rc = check_launch("bwd_preprocess_kernel")) != FA_OK) return rc;
+  {
+    // d / 8 threads per row, 256 threads per block
+    const long long pre_threads = static_cast<long long>(BH) * ws.n_pad * (d / 8);
+    const unsigned blocks = static_cast<unsigned>((pre_threads + 255) / 256);
+    auto* pre = d == 64 ? fa::bwd_preprocess_kernel<64> : fa::bwd_preprocess_kernel<128>;
+    pre<<<blocks, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse,
+        reinterpret_cast<float*>(wsb + ws.lse2), reinterpret_cast<float*>(wsb + ws.dvec),
+        deterministic ? nullptr : reinterpret_cast<float*>(wsb + ws.dq), BH, N, ws.n_pad);
+    if ((rc = check_launch("bwd_preprocess_kernel")) != FA_OK) return rc;
+  }
   if (deterministic) {
     // dK and dV by the dK/dV kernel, dQ by the query-stationary kernel: no atomics
     if (d == 64)

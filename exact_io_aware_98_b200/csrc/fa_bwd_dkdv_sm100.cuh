@@ -109,8 +109,16 @@ fa_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int lane = threadIdx.x & 31;
   const int G = p.H / p.H_kv;                          // query heads per K/V head
   const int BHkv = p.B * p.H_kv;
-  const int jt = static_cast<int>(blockIdx.x) / BHkv;  // KV tile; small jt (most work) first
-  const int bhk = static_cast<int>(blockIdx.x) % BHkv;  // (b, K/V head)
+  // CTA order: groups of p.hgroup K/V heads in turn (a group's Q and dO fit in half of L2, so
+  // the re-reads of Q and dO by the KV tiles of a head hit L2), and inside a group the KV tiles
+  // with the most query tiles (small jt) first.
+  const int per_group = p.hgroup * p.n_ktiles;
+  const int grp = static_cast<int>(blockIdx.x) / per_group;
+  const int g0 = grp * p.hgroup;
+  const int gn = min(p.hgroup, BHkv - g0);              // heads in this group (the last may have fewer)
+  const int rr = static_cast<int>(blockIdx.x) - grp * per_group;
+  const int jt = rr / gn;                               // KV tile
+  const int bhk = g0 + rr % gn;                         // (b, K/V head)
   const int b = bhk / p.H_kv;
   const int bhq0 = b * p.H + (bhk % p.H_kv) * G;       // first query head of the group
   const int N = p.N;

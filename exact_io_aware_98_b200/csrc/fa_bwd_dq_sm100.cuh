@@ -42,6 +42,7 @@ struct BwdDqParams {
   __nv_bfloat16* dq;          // [B*H][N][D]
   int B, H, H_kv, N, N_pad;
   int n_mtiles;               // ceil(N / 128)
+  int hgroup;                 // query heads per CTA-order group (>= 1; B*H: one group)
   float scale, scale2;
   int causal;
 };
@@ -106,8 +107,16 @@ fa_bwd_dq_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int BH = p.B * p.H;
-  const int mt = p.n_mtiles - 1 - static_cast<int>(blockIdx.x) / BH;  // heaviest tiles first
-  const int bh = static_cast<int>(blockIdx.x) % BH;
+  // CTA order: groups of p.hgroup query heads in turn (the K and V the group reads fit in half
+  // of L2, so the query tiles of a head re-read them from L2), and inside a group the heaviest
+  // query tiles (the last rows under a causal mask) first.
+  const int per_group = p.hgroup * p.n_mtiles;
+  const int grp = static_cast<int>(blockIdx.x) / per_group;
+  const int g0 = grp * p.hgroup;
+  const int gn = min(p.hgroup, BH - g0);                // heads in this group (the last may have fewer)
+  const int rr = static_cast<int>(blockIdx.x) - grp * per_group;
+  const int mt = p.n_mtiles - 1 - rr / gn;
+  const int bh = g0 + rr % gn;
   const int b = bh / p.H;
   const int bh_kv = b * p.H_kv + (bh % p.H) / (p.H / p.H_kv);  // K/V head of this query head
   const int N = p.N;

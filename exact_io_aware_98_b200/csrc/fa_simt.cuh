@@ -227,30 +227,48 @@ naive_pv_kernel(const __nv_bfloat16* __restrict__ pm, const __nv_bfloat16* __res
 // ---------------------------------------------------------------------------- backward helpers
 // Dvec_i = sum_c dO_ic O_ic (fp32); lse2_i = lse_i * log2(e) (+inf for rows with no key and for
 // the padding rows N..N_pad-1); zeroes the fp32 dQ accumulator unless dq_acc is null (the
-// deterministic backward has none).  One warp per row of N_pad.
+// deterministic backward has none).  HBM-bound: each thread takes 8 consecutive elements of a
+// row (16-byte loads of O and dO, 32-byte stores of zeros), D/8 threads per row, the row's dot
+// product reduced over those lanes.  D is 64 or 128.
+template <int D>
 __global__ void __launch_bounds__(256)
 bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
                       const float* __restrict__ lse, float* __restrict__ lse2,
                       float* __restrict__ dvec, float* __restrict__ dq_acc, int BH, int N,
-                      int N_pad, int d) {
-  const long long r = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (r >= static_cast<long long>(BH) * N_pad) return;
+                      int N_pad) {
+  constexpr int T = D / 8;  // threads per row
+  const long long r = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) / T;
+  const int part = threadIdx.x % T;
+  if (r >= static_cast<long long>(BH) * N_pad) return;  // whole row groups leave together
   const int bh = static_cast<int>(r / N_pad), i = static_cast<int>(r % N_pad);
   if (i >= N) {
-    if (lane == 0) {
+    if (part == 0) {
       lse2[r] = INFINITY;
       dvec[r] = 0.f;
     }
     return;
   }
-  const size_t off = (static_cast<size_t>(bh) * N + i) * d;
+  const size_t off = (static_cast<size_t>(bh) * N + i) * D + part * 8;
+  const uint4 a = *reinterpret_cast<const uint4*>(o + off);
+  const uint4 g = *reinterpret_cast<const uint4*>(dO + off);
+  const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
   float acc = 0.f;
-  for (int c = lane; c < d; c += 32) acc = fmaf(__bfloat162float(dO[off + c]), __bfloat162float(o[off + c]), acc);
-  for (int offs = 16; offs > 0; offs >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, offs);
-  if (dq_acc != nullptr)
-    for (int c = lane; c < d; c += 32) dq_acc[off + c] = 0.f;
-  if (lane == 0) {
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    acc = fmaf(__uint_as_float(gw[e] << 16), __uint_as_float(aw[e] << 16), acc);
+    acc = fmaf(__uint_as_float(gw[e] & 0xffff0000u), __uint_as_float(aw[e] & 0xffff0000u), acc);
+  }
+  // the T lanes of this row (aligned within the warp; other rows' lanes may have returned)
+  const unsigned lane = threadIdx.x & 31u;
+  const unsigned group = ((T == 32) ? 0xffffffffu : ((1u << T) - 1u)) << (lane & ~(T - 1u));
+#pragma unroll
+  for (int offs = T / 2; offs > 0; offs >>= 1) acc += __shfl_xor_sync(group, acc, offs);
+  if (dq_acc != nullptr) {
+    float4* z = reinterpret_cast<float4*>(dq_acc + off);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  if (part == 0) {
     const float ls = lse[static_cast<size_t>(bh) * N + i];
     lse2[r] = (ls == -INFINITY) ? INFINITY : ls * 1.4426950408889634f;
     dvec[r] = acc;
