@@ -18,6 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfa.so")
 
 FA_BF16, FA_F32 = 0, 1
+BWD_DKDV_PAIR, BWD_DKDV_SINGLE = 1, 2   # fa.h FA_BWD_DKDV_*
 _STATUS = {0: "FA_OK", -1: "FA_ERR_INVALID", -2: "FA_ERR_UNSUPPORTED", -3: "FA_ERR_ALIGN",
            -4: "FA_ERR_CUDA", -5: "FA_ERR_TIMEOUT", -6: "FA_ERR_WORKSPACE"}
 
@@ -35,6 +36,8 @@ SIGNATURES = {
                     _vp, _i, _vp, _sz, _vp]),
     "fa_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
                             _vp, _vp, _i, _vp]),
+    "fa_bwd_deterministic_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                     _i, _f, _i, _vp, _vp, _i, _vp, _sz, _i, _vp]),
     "fa_fwd_tile_reference": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp,
                                    _i, _i, _vp]),
     "fa_naive_workspace_size": (_sz, [_i, _i, _i]),
@@ -186,10 +189,12 @@ def _bwd_operands(q, k, v, o, lse, do, dq, dk, dv):
 
 def bwd(q, k, v, o, lse, do, scale: Optional[float] = None, causal: bool = False,
         block_mask=None, kv_len=None, workspace=None, dq=None, dk=None, dv=None,
-        deterministic: bool = False):
+        deterministic: bool = False, dkdv_pair: Optional[bool] = None):
     """dQ, dK, dV = fa_bwd(...); tensors on the GPU, q/o/do [B, H, N, d], k/v and dK/dV
     [B, H_kv, N, d] (fa_bwd_gqa when H_kv < H).  ``deterministic`` calls fa_bwd_deterministic:
-    bit-reproducible gradients, dQ without atomics."""
+    bit-reproducible gradients, dQ without atomics; with it, ``dkdv_pair`` True / False picks
+    the 2-CTA or the single-CTA dK/dV kernel at d = 128 (fa_bwd_deterministic_ex), None the
+    library's default."""
     lib = load()
     B, H, N, d = q.shape
     H_kv, dq, dk, dv = _bwd_operands(q, k, v, o, lse, do, dq, dk, dv)
@@ -198,7 +203,14 @@ def bwd(q, k, v, o, lse, do, scale: Optional[float] = None, causal: bool = False
     _require(ws, "workspace", torch.uint8)
     bm, kl = _masks(block_mask, kv_len)
     s = default_scale(d) if scale is None else float(scale)
-    if deterministic:
+    if deterministic and dkdv_pair is not None:
+        opt = BWD_DKDV_PAIR if dkdv_pair else BWD_DKDV_SINGLE
+        rc = lib.fa_bwd_deterministic_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do),
+                                         _ptr(dq), _ptr(dk), _ptr(dv), B, H, H_kv, N, d, s,
+                                         int(causal), bm, kl, _dtype_code(q), _ptr(ws),
+                                         ws.numel(), opt, _stream())
+        _check(rc, "fa_bwd_deterministic_ex")
+    elif deterministic:
         rc = lib.fa_bwd_deterministic(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do),
                                       _ptr(dq), _ptr(dk), _ptr(dv), B, H, H_kv, N, d, s,
                                       int(causal), bm, kl, _dtype_code(q), _ptr(ws), ws.numel(),

@@ -13,6 +13,7 @@
 #include <vector>
 
 #include "fa.h"
+#include "fa_bwd_dkdv_pair_sm100.cuh"
 #include "fa_bwd_dkdv_sm100.cuh"
 #include "fa_bwd_dq_sm100.cuh"
 #include "fa_bwd_sm100.cuh"
@@ -311,6 +312,55 @@ int launch_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
   return check_launch("fa_bwd_dkdv_sm100_kernel");
 }
 
+// dK and dV at d = 128 on CTA pairs with 2-CTA MMAs (fa_bwd_dkdv_pair_sm100.cuh); the same sums
+// in the same order as launch_bwd_dkdv<128>.
+int launch_bwd_dkdv_pair(const void* q, const void* k, const void* v, const void* dO, void* dk,
+                         void* dv, int B, int H, int H_kv, int N, float scale, int causal,
+                         const uint8_t* bm, const int32_t* kv_len, const BwdWs& ws, uint8_t* wsb,
+                         cudaStream_t stream) {
+  using L = fa::BwdPairLayout;
+  constexpr int D = L::D;
+  CUtensorMap mq, mk, mv, mdo;
+  const int BH = B * H;
+  int rc;
+  if ((rc = make_map(&mq, q, BH, N, D, 64, "q")) != FA_OK) return rc;
+  if ((rc = make_map(&mk, k, B * H_kv, N, D, 128, "k")) != FA_OK) return rc;
+  if ((rc = make_map(&mv, v, B * H_kv, N, D, 128, "v")) != FA_OK) return rc;
+  if ((rc = make_map(&mdo, dO, BH, N, D, 64, "dO")) != FA_OK) return rc;
+  if ((rc = set_smem(fa::fa_bwd_dkdv_pair_sm100_kernel, L::SMEM_ALLOC)) != FA_OK) return rc;
+  fa::BwdParams p;
+  p.block_mask = bm;
+  p.kv_len = kv_len;
+  p.lse2 = reinterpret_cast<const float*>(wsb + ws.lse2);
+  p.dvec = reinterpret_cast<const float*>(wsb + ws.dvec);
+  p.dq_acc = nullptr;
+  {
+    // K/V heads per CTA-order group: the group's Q and dO, 4 bytes per element of its G query
+    // heads, within half of the 126 MB L2.
+    const long long per_head = 4ll * (H / H_kv) * N * D;
+    p.hgroup = static_cast<int>(
+        std::max(1ll, std::min((64ll << 20) / per_head, static_cast<long long>(B) * H_kv)));
+  }
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.B = B;
+  p.H = H;
+  p.H_kv = H_kv;
+  p.N = N;
+  p.N_pad = ws.n_pad;
+  p.n_ktiles = (N + 127) / 128;
+  p.scale = scale;
+  p.scale2 = scale * kLog2e;
+  p.causal = causal ? 1 : 0;
+  // two CTAs (one cluster) per pair of KV tiles
+  const long long grid = 2ll * ((p.n_ktiles + 1) / 2) * B * H_kv;
+  if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
+  TimedLaunch tl("fa_bwd_dkdv_pair_sm100_kernel", stream);
+  fa::fa_bwd_dkdv_pair_sm100_kernel<<<static_cast<unsigned>(grid), 320, L::SMEM_ALLOC, stream>>>(
+      mq, mk, mv, mdo, p);
+  return check_launch("fa_bwd_dkdv_pair_sm100_kernel");
+}
+
 // dQ without atomics: one CTA per 128 query rows walks the KV tiles (fa_bwd_dq_sm100.cuh).
 template <int D>
 int launch_bwd_dq(const void* q, const void* k, const void* v, const void* dO, void* dq, int B,
@@ -405,6 +455,14 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   return fail(FA_ERR_INVALID, "unknown dtype %d", dtype);
 }
 
+// fa_bwd_deterministic_ex options: which dK/dV kernel runs at d = 128.
+constexpr bool kPairDkdvDefault = false;  // measured slower (see the kernel header)
+bool use_pair_dkdv(int options) {
+  if (options & FA_BWD_DKDV_SINGLE) return false;
+  if (options & FA_BWD_DKDV_PAIR) return true;
+  return kPairDkdvDefault;
+}
+
 // Argument checks shared by every backward entry point (everything but the workspace).
 int bwd_checks(const void* q, const void* k, const void* v, const void* o, const float* lse,
                const void* dO, const void* dq, const void* dk, const void* dv, int B, int H,
@@ -427,7 +485,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
              const void* dO, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N, int d,
              float scale, int causal, const uint8_t* block_mask, const int32_t* kv_len,
              int dtype, void* workspace, size_t workspace_bytes, void* stream,
-             bool deterministic) {
+             bool deterministic, int options = 0) {
   int rc = bwd_checks(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, scale, dtype);
   if (rc != FA_OK) return rc;
   const BwdWs ws = bwd_ws(B, H, N, d);
@@ -469,9 +527,12 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     if ((rc = check_launch("bwd_preprocess_kernel")) != FA_OK) return rc;
   }
   if (deterministic) {
-    // dK and dV by the dK/dV kernel, dQ by the query-stationary kernel: no atomics
+    // dK and dV by the dK/dV kernel, dQ by the query-stationary kernel: no atomics.  At d = 128
+    // the dK/dV kernel runs on CTA pairs (2-CTA MMAs) unless the caller asks for one CTA.
     if (d == 64)
       rc = launch_bwd_dkdv<64>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
+    else if (use_pair_dkdv(options))
+      rc = launch_bwd_dkdv_pair(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
     else
       rc = launch_bwd_dkdv<128>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
     if (rc != FA_OK) return rc;
@@ -537,6 +598,18 @@ int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void
                          void* workspace, size_t workspace_bytes, void* stream) {
   return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, scale, causal, block_mask,
                   kv_len, dtype, workspace, workspace_bytes, stream, true);
+}
+
+int fa_bwd_deterministic_ex(const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
+                            int H, int H_kv, int N, int d, float scale, int causal,
+                            const uint8_t* block_mask, const int32_t* kv_len, int dtype,
+                            void* workspace, size_t workspace_bytes, int options, void* stream) {
+  if ((options & ~(FA_BWD_DKDV_PAIR | FA_BWD_DKDV_SINGLE)) != 0 ||
+      (options & (FA_BWD_DKDV_PAIR | FA_BWD_DKDV_SINGLE)) == (FA_BWD_DKDV_PAIR | FA_BWD_DKDV_SINGLE))
+    return fail(FA_ERR_INVALID, "unknown or contradictory backward options 0x%x", options);
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, H, H_kv, N, d, scale, causal, block_mask,
+                  kv_len, dtype, workspace, workspace_bytes, stream, true, options);
 }
 
 int fa_fwd_tile_reference(const void* q, const void* k, const void* v, void* o, float* lse,

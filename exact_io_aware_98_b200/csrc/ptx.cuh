@@ -357,6 +357,138 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ----------------------------------------------------------------------------- CTA pairs
+// A cluster of two CTAs whose tensor cores work as one (tcgen05 cta_group::2): the even CTA
+// (rank 0, the leader) issues the MMAs, each CTA supplies half of every operand from its own
+// shared memory or TMEM and receives its half of the accumulator in its own TMEM.
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The shared::cluster address of the variable at `local` in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void* local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+}
+// Arrive on an mbarrier anywhere in the cluster, releasing this thread's prior writes at
+// cluster scope.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+               : "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr_, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr_), "r"(v) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// mbar_wait with acquire at cluster scope (for barriers that the other CTA of the pair arrives
+// on, or that its MMAs complete), bounded in the same way.
+__device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                             int site) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 15u) == 0u) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        atomicCAS(&g_status, 0u, (static_cast<unsigned>(site) << 16) | (blockIdx.x & 0xffffu));
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+// mbar_wait_drain with acquire at cluster scope.
+__device__ __forceinline__ bool mbar_wait_drain_cl(uint64_t* bar, uint32_t parity, int site) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 15u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicCAS(&g_status, 0u, (static_cast<unsigned>(site) << 16) | (blockIdx.x & 0xffffu));
+      return false;
+    }
+  }
+}
+// TMA tile load into this CTA's shared memory whose completion is counted on an mbarrier of
+// either CTA of the pair (`cluster_bar`, a shared::cluster address).  No multicast.
+__device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const CUtensorMap* map,
+                                                 uint32_t cluster_bar, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(cluster_bar)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+// Pair versions of the warp-collective four-MMA issue (leader CTA only): D (+)= A_i * B_i with
+// M = 256 across the pair.
+__device__ __forceinline__ void mma2_ss_x4(uint32_t d_tmem, const uint64_t (&a)[4],
+                                           const uint64_t (&b)[4], uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "elect.sync _|q, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %10, 0;\n\t"
+      "@q tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %9, p;\n\t"
+      "@q tcgen05.mma.cta_group::2.kind::f16 [%0], %3, %4, %9, 1;\n\t"
+      "@q tcgen05.mma.cta_group::2.kind::f16 [%0], %5, %6, %9, 1;\n\t"
+      "@q tcgen05.mma.cta_group::2.kind::f16 [%0], %7, %8, %9, 1;\n\t}\n" ::"r"(d_tmem),
+      "l"(a[0]), "l"(b[0]), "l"(a[1]), "l"(b[1]), "l"(a[2]), "l"(b[2]), "l"(a[3]), "l"(b[3]),
+      "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma2_ts_x4(uint32_t d_tmem, const uint32_t (&a)[4],
+                                           const uint64_t (&b)[4], uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "elect.sync _|q, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %10, 0;\n\t"
+      "@q tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %9, p;\n\t"
+      "@q tcgen05.mma.cta_group::2.kind::f16 [%0], [%3], %4, %9, 1;\n\t"
+      "@q tcgen05.mma.cta_group::2.kind::f16 [%0], [%5], %6, %9, 1;\n\t"
+      "@q tcgen05.mma.cta_group::2.kind::f16 [%0], [%7], %8, %9, 1;\n\t}\n" ::"r"(d_tmem),
+      "r"(a[0]), "l"(b[0]), "r"(a[1]), "l"(b[1]), "r"(a[2]), "l"(b[2]), "r"(a[3]), "l"(b[3]),
+      "r"(idesc), "r"(acc)
+      : "memory");
+}
+// Warp-collective commit of the pair's MMAs to an mbarrier anywhere in the cluster.
+__device__ __forceinline__ void mma2_commit_w(uint32_t cluster_bar) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "elect.sync _|q, 0xffffffff;\n\t"
+      "@q tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(
+          cluster_bar)
+      : "memory");
+}
+
 // ----------------------------------------------------------------------------- math helpers
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

@@ -153,6 +153,31 @@ int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void
                          const uint8_t* block_mask, const int32_t* kv_len, int dtype,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* Options of fa_bwd_deterministic_ex (bits; 0 = the library's default). */
+enum {
+  FA_BWD_DKDV_PAIR = 1,   /* d = 128: dK and dV on pairs of CTAs with 2-CTA MMAs */
+  FA_BWD_DKDV_SINGLE = 2  /* d = 128: dK and dV with one CTA per 128 keys (default) */
+};
+
+/*
+ * fa_bwd_deterministic_ex -- fa_bwd_deterministic with a choice of dK/dV kernel at d = 128
+ * (`options`, FA_BWD_DKDV_*; ignored at d = 64 and for FA_F32).  Both kernels sum every dK and
+ * dV element over the same terms in the same order.
+ *   FA_BWD_DKDV_PAIR: a cluster of two CTAs owns 256 keys and the even CTA issues tcgen05 MMAs
+ *     with cta_group::2 (M = 256 keys, each CTA holding its 128 keys' K, V and accumulators); Q
+ *     and dO are loaded in halves (query rows for the scores, head-dimension columns for the
+ *     gradients), so each SM's tensor core reads half of every B operand from its own shared
+ *     memory.  Every tile load is a plain TMA load of this GPU's memory (no multicast).
+ *   FA_BWD_DKDV_SINGLE: one CTA per 128 keys with cta_group::1 MMAs.
+ * Setting both bits, or any other bit, gives FA_ERR_INVALID.  Everything else is as for
+ * fa_bwd_deterministic.
+ */
+int fa_bwd_deterministic_ex(const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
+                            int H, int H_kv, int N, int d, float scale, int causal,
+                            const uint8_t* block_mask, const int32_t* kv_len, int dtype,
+                            void* workspace, size_t workspace_bytes, int options, void* stream);
+
 /* Flags of fa_fwd_tile_reference: the other two axes of the deviation study. */
 enum {
   FA_TILE_REVERSE = 1,    /* visit the key tiles from the last to the first */
@@ -211,7 +236,8 @@ int fa_diag_wait_timeout(int site, void* stream);
  *                            counted).
  *   fa_kernel_timing      -- enable != 0: from now on every launch of a tensor-core kernel
  *                            (fa_fwd_sm100_kernel, fa_bwd_sm100_kernel, fa_bwd_dkdv_sm100_kernel,
- *                            fa_bwd_dq_sm100_kernel) is bracketed by two CUDA events recorded on
+ *                            fa_bwd_dkdv_pair_sm100_kernel, fa_bwd_dq_sm100_kernel) is
+ *                            bracketed by two CUDA events recorded on
  *                            the launch's stream; enable == 0 stops recording.  Off by default.
  *   fa_kernel_timing_read -- waits for the recorded launches of every kernel whose name contains
  *                            `name` ("" = all), stores how many there were in *launches and the

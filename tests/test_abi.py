@@ -155,3 +155,12 @@ def test_measurement_diagnostics_without_a_gpu(lib):
     assert n.value == 0 and ms.value == 0.0
     assert lib.fa_kernel_timing(0) == OK
     assert lib.fa_kernel_timing_read(b"fa_", None, ctypes.byref(ms)) == INVALID
+
+
+def test_deterministic_ex_rejects_unknown_options(lib):
+    """Unknown option bits, or both dK/dV kernels at once, are refused before any launch."""
+    for opt in (3, 4, 1 << 30):
+        rc = lib.fa_bwd_deterministic_ex(A, A, A, A, A, A, A, A, A, 1, 2, 2, 256, 128, 0.088,
+                                         1, None, None, 0, A, 1 << 20, opt, None)
+        assert rc == INVALID
+        assert "option" in lib.fa_get_last_error().decode()
