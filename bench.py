@@ -519,7 +519,10 @@ def cpu_baseline_leg(args, x, o, lse, dq):
 
 def deviation_sweep():
     """Numeric deviation vs the FP64 golden across key-tile widths, next to the naive kernel
-    (the microbenchmark of "Is Flash Attention Stable?"), on 32 heads of the padding workload."""
+    (the microbenchmark of "Is Flash Attention Stable?"), on 32 heads of the padding workload.
+    Each variant is measured on its bf16 output and, beside it, on the fp32 O/l before that
+    rounding: the bf16 cast alone contributes up to half an ulp of O, which would otherwise hide
+    the effect of the tile width."""
     import oracle
     import exact_io_aware_98_b200 as fa
     x = syn.workload_inputs("bert_padding", with_grad=False, H=2)
@@ -530,24 +533,31 @@ def deviation_sweep():
     def stat(t):
         e = np.abs(t.float().cpu().double().numpy() - gold)
         return {"max": float(e.max()), "mean": float(e.mean())}
-    kw = dict(scale=g["scale"], kv_len=g["kv_len"])
-    o_tc, _ = fa.fwd(g["q"], g["k"], g["v"], **kw)
-    out["tcgen05_Br128_Bc128_lazy"] = stat(o_tc)
-    # the study's axes: key-tile width Bc, the order the key tiles are visited in, and whether
-    # the normaliser l sums the fp32 P or the bf16-rounded P that enters P.V
+
+    def both(**kw_tile):
+        o, _ = fa.fwd_tile_reference(g["q"], g["k"], g["v"], scale=g["scale"], kv_len=g["kv_len"],
+                                     **kw_tile)
+        o32, _ = fa.fwd_tile_reference(g["q"], g["k"], g["v"], scale=g["scale"],
+                                       kv_len=g["kv_len"], o_f32=True, **kw_tile)
+        return {"bf16": stat(o), "fp32_before_cast": stat(o32)}
+    # the tensor-core forward itself at two key-tile widths (64 is the library's d = 64 kernel)
+    for bc in (64, 128):
+        out[f"tcgen05_Br128_Bc{bc}_lazy"] = both(bc=bc, tensor_core=True)
+    # the study's axes on the CUDA-core reference: key-tile width Bc, the order the key tiles are
+    # visited in, and whether the normaliser l sums the fp32 P or the bf16-rounded P
     for bc in (64, 128, 256):
         for reverse in (False, True):
             for l_rounded in (False, True):
-                o_t, _ = fa.fwd_tile_reference(g["q"], g["k"], g["v"], bc, reverse=reverse,
-                                               l_rounded=l_rounded, **kw)
                 key = f"tile_Bc{bc}_{'reverse' if reverse else 'forward'}_l{'bf16' if l_rounded else 'fp32'}"
-                out[key] = stat(o_t)
+                out[key] = both(bc=bc, reverse=reverse, l_rounded=l_rounded)
+    kw = dict(scale=g["scale"], kv_len=g["kv_len"])
     o_n, _ = fa.naive_fwd(g["q"], g["k"], g["v"], **kw)
-    out["naive_materialised"] = stat(o_n)
+    out["naive_materialised"] = {"bf16": stat(o_n)}
+    o_tc, _ = fa.fwd(g["q"], g["k"], g["v"], **kw)
     diff = (o_tc.float() - o_n.float()).abs()
     out["tcgen05_vs_naive"] = {"max": float(diff.max()), "mean": float(diff.mean())}
     out["note"] = ("row-wise arithmetic does not depend on Br (query-tile height), so the sweep "
-                   "varies Bc; the tcgen05 kernel is Br=Bc=128 with a lazy (2^8) rescale")
+                   "varies Bc; the tcgen05 kernel is Br=128 with a lazy (2^8) rescale")
     return out
 
 

@@ -251,27 +251,31 @@ def bwd_noalloc(q, k, v, o, lse, do, scale: Optional[float] = None, causal: bool
     return dq, dk, dv
 
 
-TILE_REVERSE = 1     # fa.h FA_TILE_REVERSE: key tiles visited last to first
-TILE_L_ROUNDED = 2   # fa.h FA_TILE_L_ROUNDED: l sums the bf16-rounded P
+TILE_REVERSE = 1          # fa.h FA_TILE_REVERSE: key tiles visited last to first
+TILE_L_ROUNDED = 2        # fa.h FA_TILE_L_ROUNDED: l sums the bf16-rounded P
+TILE_TENSOR_CORE = 4      # fa.h FA_TILE_TENSOR_CORE: the tcgen05 forward with bc-key tiles
+TILE_O_F32 = 8            # fa.h FA_TILE_O_F32: fp32 O/l before its bf16 rounding
 
 
 def fwd_tile_reference(q, k, v, bc: int, scale: Optional[float] = None, causal: bool = False,
                        block_mask=None, kv_len=None, reverse: bool = False,
-                       l_rounded: bool = False):
-    """bf16 CUDA-core forward that rescales after every `bc` keys (deviation study); `reverse`
-    visits the key tiles last to first, `l_rounded` sums l over the bf16-rounded P."""
+                       l_rounded: bool = False, tensor_core: bool = False, o_f32: bool = False):
+    """bf16 forward that rescales after every `bc` keys (deviation study): the CUDA-core
+    reference (`reverse` visits the key tiles last to first, `l_rounded` sums l over the
+    bf16-rounded P) or, with `tensor_core`, the tcgen05 forward with bc-key tiles (d = 64,
+    bc 64 or 128).  `o_f32` returns the fp32 O/l before its bf16 rounding."""
     lib = load()
     B, H, N, d = q.shape
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _require(t, n, torch.bfloat16)
-    o = torch.empty_like(q)
+    o = torch.empty(q.shape, dtype=torch.float32 if o_f32 else torch.bfloat16, device=q.device)
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     bm, kl = _masks(block_mask, kv_len)
     s = default_scale(d) if scale is None else float(scale)
+    flags = ((TILE_REVERSE if reverse else 0) | (TILE_L_ROUNDED if l_rounded else 0) |
+             (TILE_TENSOR_CORE if tensor_core else 0) | (TILE_O_F32 if o_f32 else 0))
     rc = lib.fa_fwd_tile_reference(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, H, N, d, s,
-                                   int(causal), bm, kl, int(bc),
-                                   (TILE_REVERSE if reverse else 0) |
-                                   (TILE_L_ROUNDED if l_rounded else 0), _stream())
+                                   int(causal), bm, kl, int(bc), flags, _stream())
     _check(rc, "fa_fwd_tile_reference")
     return o, l
 

@@ -182,22 +182,24 @@ BwdWs bwd_ws(int B, int H, int N, int d) {
   return w;
 }
 
-template <int D>
+// BN: keys per KV tile; O32: o is fp32 O/l (deviation study) instead of bf16 O.
+template <int D, int BN = fa::fwd_bn<D>(), bool O32 = false>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                int H_kv, int N, float scale, int causal, const uint8_t* bm,
                const int32_t* kv_len, cudaStream_t stream) {
-  using L = fa::FwdLayout<D>;
+  using L = fa::FwdLayout<D, BN>;
   CUtensorMap mq, mk, mv;
   const int BH = B * H;
   int rc;
   if ((rc = make_map(&mq, q, BH, N, D, 128, "q")) != FA_OK) return rc;
   if ((rc = make_map(&mk, k, B * H_kv, N, D, L::BN, "k")) != FA_OK) return rc;
   if ((rc = make_map(&mv, v, B * H_kv, N, D, L::BN, "v")) != FA_OK) return rc;
-  if ((rc = set_smem(fa::fa_fwd_sm100_kernel<D>, L::SMEM_ALLOC)) != FA_OK) return rc;
+  if ((rc = set_smem(fa::fa_fwd_sm100_kernel<D, BN, O32>, L::SMEM_ALLOC)) != FA_OK) return rc;
   fa::FwdParams p;
   p.block_mask = bm;
   p.kv_len = kv_len;
-  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o = O32 ? nullptr : static_cast<__nv_bfloat16*>(o);
+  p.o32 = O32 ? static_cast<float*>(o) : nullptr;
   p.lse = lse;
   p.B = B;
   p.H = H;
@@ -213,7 +215,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   const long long grid = static_cast<long long>(p.n_mtiles) * BH;
   if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
   TimedLaunch tl("fa_fwd_sm100_kernel", stream);
-  fa::fa_fwd_sm100_kernel<D><<<static_cast<unsigned>(grid), 320, L::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
+  fa::fa_fwd_sm100_kernel<D, BN, O32><<<static_cast<unsigned>(grid), 320, L::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
   return check_launch("fa_fwd_sm100_kernel");
 }
 
@@ -449,7 +451,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     fa::fa_fwd_rowwarp_kernel<float, false><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
         static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
         static_cast<float*>(o), lse, block_mask, kv_len, B, H, N, d, scale, causal ? 1 : 0, 128, 0,
-        H_kv);
+        H_kv, nullptr);
     return check_launch("fa_fwd_rowwarp_kernel<f32>");
   }
   return fail(FA_ERR_INVALID, "unknown dtype %d", dtype);
@@ -619,15 +621,30 @@ int fa_fwd_tile_reference(const void* q, const void* k, const void* v, void* o, 
   int rc = common_checks(q, k, v, o, lse, B, H, N, d, scale);
   if (rc != FA_OK) return rc;
   if (d > 128) return fail(FA_ERR_UNSUPPORTED, "d <= 128 required, got %d", d);
-  if (bc < 32 || bc > 256 || (bc % 32) != 0) return fail(FA_ERR_INVALID, "bc must be 32..256 in steps of 32");
-  if ((flags & ~(FA_TILE_REVERSE | FA_TILE_L_ROUNDED)) != 0)
+  if ((flags & ~(FA_TILE_REVERSE | FA_TILE_L_ROUNDED | FA_TILE_TENSOR_CORE | FA_TILE_O_F32)) != 0)
     return fail(FA_ERR_INVALID, "unknown tile-reference flags 0x%x", flags);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool o32 = (flags & FA_TILE_O_F32) != 0;
+  if (flags & FA_TILE_TENSOR_CORE) {
+    // the tcgen05 forward itself, with bc-key tiles (its own lazy rescale and fp32-P normaliser)
+    if (flags & (FA_TILE_REVERSE | FA_TILE_L_ROUNDED))
+      return fail(FA_ERR_INVALID, "the tensor-core forward has no reverse or rounded-l variant");
+    if (d != 64 || (bc != 64 && bc != 128))
+      return fail(FA_ERR_UNSUPPORTED, "tensor-core tile sweep: d = 64 and bc in {64, 128}");
+    if (bc == 64)
+      return o32 ? launch_fwd<64, 64, true>(q, k, v, o, lse, B, H, H, N, scale, causal, block_mask, kv_len, s)
+                 : launch_fwd<64, 64, false>(q, k, v, o, lse, B, H, H, N, scale, causal, block_mask, kv_len, s);
+    return o32 ? launch_fwd<64, 128, true>(q, k, v, o, lse, B, H, H, N, scale, causal, block_mask, kv_len, s)
+               : launch_fwd<64, 128, false>(q, k, v, o, lse, B, H, H, N, scale, causal, block_mask, kv_len, s);
+  }
+  if (bc < 32 || bc > 256 || (bc % 32) != 0) return fail(FA_ERR_INVALID, "bc must be 32..256 in steps of 32");
   const long long rows = static_cast<long long>(B) * H * N;
   fa::fa_fwd_rowwarp_kernel<__nv_bfloat16, true>
-      <<<static_cast<unsigned>((rows + 7) / 8), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      <<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
           static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-          static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), lse, block_mask,
-          kv_len, B, H, N, d, scale, causal ? 1 : 0, bc, flags, H);
+          static_cast<const __nv_bfloat16*>(v), o32 ? nullptr : static_cast<__nv_bfloat16*>(o),
+          lse, block_mask, kv_len, B, H, N, d, scale, causal ? 1 : 0, bc, flags, H,
+          o32 ? static_cast<float*>(o) : nullptr);
   return check_launch("fa_fwd_rowwarp_kernel<bf16>");
 }
 

@@ -47,6 +47,7 @@ struct FwdParams {
   const uint8_t* block_mask;  // [nb][nb] (nb = ceil(N/128)) or nullptr
   const int32_t* kv_len;      // [B] or nullptr
   __nv_bfloat16* o;           // [B*H][N][D]
+  float* o32;                 // [B*H][N][D] fp32 O/l, written instead of o by the O32 variant
   float* lse;                 // [B*H][N]
   int B, H, N;
   int H_kv;                   // K/V heads; query head h reads K/V head h / (H / H_kv)
@@ -56,13 +57,18 @@ struct FwdParams {
   int causal;
 };
 
+// Key-tile width: fwd_bn<D> keys per KV tile in the library's forward; the deviation study
+// also runs d = 64 with 128-key tiles.
 template <int D>
+constexpr int fwd_bn() { return D == 64 ? 64 : 128; }
+
+template <int D, int BN_ = fwd_bn<D>()>
 struct FwdLayout {
   static constexpr int BM = 128;                    // query rows per Q tile
-  static constexpr int BN = D == 64 ? 64 : 128;     // keys per KV tile
-  static constexpr int CTAS_PER_SM = D == 64 ? 2 : 1;
-  static constexpr int KST = D == 64 ? 4 : 3;       // K ring depth
-  static constexpr int VST = D == 64 ? 4 : 2;       // V ring depth
+  static constexpr int BN = BN_;                    // keys per KV tile
+  static constexpr int CTAS_PER_SM = BN == 64 ? 2 : 1;
+  static constexpr int KST = BN == 64 ? 4 : (D == 64 ? 5 : 3);  // K ring depth
+  static constexpr int VST = BN == 64 ? 4 : (D == 64 ? 4 : 2);  // V ring depth
   static constexpr int SUB = D / 64;                // 64-column (128-byte) sub-tiles
   static constexpr int SUBTILE = 128 * 128;         // bytes of one 128-row x 64-col Q sub-tile
   static constexpr int TILE = 128 * D * 2;          // bytes of one 128-row Q tile
@@ -73,12 +79,17 @@ struct FwdLayout {
   static constexpr int OFF_V = OFF_K + KST * KV_TILE;
   static constexpr int OFF_BAR = OFF_V + VST * KV_TILE;
   // q, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], p_full[2], o_done[2], fin
-  static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 6 + 1;
+  // P in two key halves (128-key tiles): the MMA warp issues P.V over keys 0-63 as soon as that
+  // half of P is in TMEM, while the softmax warpgroup computes the exponentials of keys 64-127
+  static constexpr bool SPLIT_P = BN == 128;
+  // q, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], p_full[2], o_done[2],
+  // p2_full[2], fin
+  static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 6 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;   // slack for 1024-byte alignment
   static_assert(CTAS_PER_SM * (SMEM_ALLOC + 1024) <= 233472, "shared memory per SM");
-  static constexpr uint32_t TMEM_COLS = D == 64 ? 256 : 512;
+  static constexpr uint32_t TMEM_COLS = 2 * BN + 2 * D <= 256 ? 256 : 512;
   static constexpr uint32_t O_COL0 = 2 * BN;
   static_assert(O_COL0 + 2 * D <= TMEM_COLS, "TMEM budget");
   // one P pair in EMU_EVERY is exponentiated on the FMA pipe (0 = all on MUFU)
@@ -93,12 +104,14 @@ enum : int {
   SITE_FWD_SM_O = 9
 };
 
-template <int D>
-__global__ void __launch_bounds__(320, FwdLayout<D>::CTAS_PER_SM)
+// O32: write the fp32 O/l to p.o32 instead of bf16 O to p.o (the deviation study's view of the
+// output before its bf16 rounding).
+template <int D, int BN_ = fwd_bn<D>(), bool O32 = false>
+__global__ void __launch_bounds__(320, FwdLayout<D, BN_>::CTAS_PER_SM)
 fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, BN_>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -111,7 +124,8 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint64_t* bar_sf = bar_ve + L::VST;
   uint64_t* bar_pf = bar_sf + 2;
   uint64_t* bar_od = bar_pf + 2;
-  uint64_t* bar_fin = bar_od + 2;
+  uint64_t* bar_p2 = bar_od + 2;          // [2] second half of P_w in TMEM (SPLIT_P)
+  uint64_t* bar_fin = bar_p2 + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -169,6 +183,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int w = 0; w < 2; ++w) {
       mbar_init(&bar_sf[w], 1);
       mbar_init(&bar_pf[w], 128);
+      mbar_init(&bar_p2[w], 128);
       mbar_init(&bar_od[w], 1);
     }
     mbar_init(bar_fin, 1);
@@ -247,6 +262,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     int cnt0 = 0, cnt1 = 0;
     int prev_flags = 0, prev_vs = 0;
     // O_w += P_w V(vs): P_w from TMEM (bf16 pairs over S_w), V MN-major.
+    // With SPLIT_P the second batch of four K-steps (keys 64-127) waits for the second half of P.
     auto issue_pv = [&](int w, int vs, int& cnt) -> bool {
       if (!mbar_wait_w(&bar_pf[w], cnt & 1, abort_flag, SITE_FWD_MMA_P)) return false;
       tc_fence_after();
@@ -255,6 +271,10 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint64_t vb = v_desc + static_cast<uint64_t>((vs * L::KV_TILE) >> 4);
 #pragma unroll
       for (int kb = 0; kb < L::BN / 64; ++kb) {
+        if (L::SPLIT_P && kb == 1) {
+          if (!mbar_wait_w(&bar_p2[w], cnt & 1, abort_flag, SITE_FWD_MMA_P)) return false;
+          tc_fence_after();
+        }
         uint32_t a[4];
         uint64_t b[4];
 #pragma unroll
@@ -372,15 +392,20 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (tmax > m_ref + 8.0f) m_new = tmax;  // also taken when m_ref is still -inf
       const float alpha = (m_new == m_ref) ? 1.0f : ex2_approx(m_ref - m_new);
       const float neg_base = (m_new == -INFINITY) ? 0.0f : -m_new;
+      const bool rescale = (cnt > 0) && (m_new != m_ref);
+      m_ref = m_new;
       // P = 2^(s*scale2 - m) in pairs: packed fp32x2 scale-and-shift and row sums (four
       // independent accumulator pairs).  On tiles without masked elements, one pair in
       // L::EMU_EVERY takes 2^x on the FMA pipe instead of MUFU, which the other pairs keep busy.
+      // P goes to TMEM (bf16 over the front of S_w) and is handed to the MMA warp in halves of
+      // the key tile with SPLIT_P, else at once.
       float ra[4] = {0.f, 0.f, 0.f, 0.f}, rb[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[NC][16];
-      auto exp_pairs = [&](bool use_fma) {
+      // chunk c (32 keys) of P; called with compile-time c so that r[c] stays in registers
+      auto exp_chunk = [&](bool use_fma, int c) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int q = 0; q < BN / 2; ++q) {
-          const int c = q >> 4, i = q & 15;
+        for (int i = 0; i < 16; ++i) {
+          const int q = 16 * c + i;
           float x0, x1, p0, p1;
           ffma2(x0, x1, __uint_as_float(r[c][2 * i]), __uint_as_float(r[c][2 * i + 1]), scale2,
                 scale2, neg_base, neg_base);
@@ -391,31 +416,55 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             p1 = ex2_approx(x1);
           }
           fadd2(ra[q & 3], rb[q & 3], ra[q & 3], rb[q & 3], p0, p1);
-          pk[c][i] = pack_bf16x2(p0, p1);
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(t_s + 16 * c, pk);
+      };
+      auto hand_over = [&](uint64_t* bar) {
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar);
+      };
+      // O rescale (rare: the reference maximum moved by more than 8), before the first P of
+      // this tile is handed over so that it precedes this tile's P.V; PV_w of the previous tile
+      // has finished (S_w of this tile was issued after it).  It runs after the first
+      // hand-over's exponentials, whose scores no longer occupy registers.
+      auto rescale_o = [&]() {
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_o + 32 * c, o);
+            tmem_ld_wait();
+            reg_fence(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(t_o + 32 * c, o);
+          }
         }
       };
-      if (edge) exp_pairs(false);  // masked elements are -inf: MUFU gives exact zeros
-      else exp_pairs(true);
-      l = alpha * l + ((ra[0] + ra[1]) + (ra[2] + ra[3]) + ((rb[0] + rb[1]) + (rb[2] + rb[3])));
+      // masked elements are -inf: MUFU gives exact zeros, so edge tiles take no FMA-pipe 2^x
+      constexpr int C1 = L::SPLIT_P ? NC / 2 : NC;  // chunks of the first hand-over
+      if (edge) {
 #pragma unroll
-      for (int c = 0; c < NC; ++c) tmem_st16(t_s + 16 * c, pk[c]);
-      const bool rescale = (cnt > 0) && (m_new != m_ref);
-      if (__any_sync(0xffffffffu, rescale)) {
+        for (int c = 0; c < C1; ++c) exp_chunk(false, c);
+      } else {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(t_o + 32 * c, o);
-          tmem_ld_wait();
-          reg_fence(o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(t_o + 32 * c, o);
-        }
+        for (int c = 0; c < C1; ++c) exp_chunk(true, c);
       }
-      m_ref = m_new;
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&bar_pf[w]);
+      rescale_o();
+      hand_over(&bar_pf[w]);
+      if constexpr (L::SPLIT_P) {
+        if (edge) {
+#pragma unroll
+          for (int c = C1; c < NC; ++c) exp_chunk(false, c);
+        } else {
+#pragma unroll
+          for (int c = C1; c < NC; ++c) exp_chunk(true, c);
+        }
+        hand_over(&bar_p2[w]);
+      }
+      l = alpha * l + ((ra[0] + ra[1]) + (ra[2] + ra[3]) + ((rb[0] + rb[1]) + (rb[2] + rb[3])));
       ++cnt;
     }
     // ---------------------------------------------------------------- epilogue: O / l, lse
@@ -427,6 +476,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       const float inv = (l > 0.f) ? 1.0f / l : 0.0f;
       __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * N + row) * D;
+      float* orow32 = p.o32 + (static_cast<size_t>(bh) * N + row) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -438,15 +488,25 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0u;
         }
-        uint32_t h[16];
+        if constexpr (O32) {
+          if (row < N) {
+            float4* dst = reinterpret_cast<float4*>(orow32 + 32 * c);
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          h[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-        if (row < N) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                                   __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+          }
+        } else {
+          uint32_t h[16];
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+          for (int i = 0; i < 16; ++i)
+            h[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+          if (row < N) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+          }
         }
       }
       if (row < N)

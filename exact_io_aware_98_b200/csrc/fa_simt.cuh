@@ -44,7 +44,8 @@ __device__ __forceinline__ bool key_allowed(int i, int j, int kvlen, int causal,
 // One warp per query row.  Keys are processed in tiles of `bc` (a multiple of 32, <= 256);
 // lane l holds the scores of keys tile0 + 32*u + l.  Output column c = 32*u + lane.
 // flags: kTileReverse visits the key tiles last to first; kTileLRounded sums l over the
-// rounded P (only meaningful with ROUND_P).
+// rounded P (only meaningful with ROUND_P).  o32 != nullptr: the fp32 O/l goes there instead of
+// the rounded O to o.
 constexpr int kTileReverse = 1;
 constexpr int kTileLRounded = 2;
 template <typename T, bool ROUND_P>
@@ -52,7 +53,7 @@ __global__ void __launch_bounds__(256)
 fa_fwd_rowwarp_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                       T* __restrict__ o, float* __restrict__ lse, const uint8_t* block_mask,
                       const int32_t* kv_len, int B, int H, int N, int d, float scale, int causal,
-                      int bc, int flags, int H_kv) {
+                      int bc, int flags, int H_kv, float* __restrict__ o32) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row_g = static_cast<long long>(blockIdx.x) * 8 + warp;  // flat bh*N + i
   if (row_g >= static_cast<long long>(B) * H * N) return;
@@ -126,7 +127,10 @@ fa_fwd_rowwarp_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
 #pragma unroll
   for (int cc = 0; cc < 4; ++cc) {
     const int c = 32 * cc + lane;
-    if (cc < ncol && c < d) o[row_g * d + c] = from_f<T>(acc[cc] * inv);
+    if (cc < ncol && c < d) {
+      if (o32 != nullptr) o32[row_g * d + c] = acc[cc] * inv;  // fp32 O/l before any rounding
+      else o[row_g * d + c] = from_f<T>(acc[cc] * inv);
+    }
   }
   if (lane == 0) lse[row_g] = (l > 0.f) ? m + logf(l) : -INFINITY;
 }

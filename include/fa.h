@@ -181,8 +181,12 @@ int fa_bwd_deterministic_ex(const void* q, const void* k, const void* v, const v
 /* Flags of fa_fwd_tile_reference: the other two axes of the deviation study. */
 enum {
   FA_TILE_REVERSE = 1,    /* visit the key tiles from the last to the first */
-  FA_TILE_L_ROUNDED = 2   /* the normaliser l sums the bf16-rounded P that enters P.V (else the
+  FA_TILE_L_ROUNDED = 2,  /* the normaliser l sums the bf16-rounded P that enters P.V (else the
                              fp32 P before rounding) */
+  FA_TILE_TENSOR_CORE = 4,/* run the tcgen05 forward itself with key tiles of bc keys (d = 64,
+                             bc in {64, 128}; not with FA_TILE_REVERSE or FA_TILE_L_ROUNDED) */
+  FA_TILE_O_F32 = 8       /* o receives the fp32 O/l, [B][H][N][d] float, before its bf16
+                             rounding (the deviation of the arithmetic without the output cast) */
 };
 
 /*
@@ -190,7 +194,8 @@ enum {
  * Flash Attention Stable?" (aibr.jp summary, sections 3-4): the running maximum and sum are
  * rescaled after every tile of `bc` keys (bc in {32, 64, ..., 256}) and P is rounded to bf16
  * before P.V, as in a tensor-core kernel with that key-tile width.  `flags` (FA_TILE_*) picks
- * the tile order and which P the normaliser sums; unknown bits give FA_ERR_INVALID.  Same
+ * the tile order and which P the normaliser sums, or swaps in the tensor-core forward itself
+ * with bc-key tiles, and whether o is written as fp32; unknown bits give FA_ERR_INVALID.  Same
  * layouts, masks and errors as fa_fwd (bf16, 1 <= d <= 128).  Not a fast path.
  */
 int fa_fwd_tile_reference(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -38,8 +38,11 @@ def test_header_declares_the_boundary():
 
 def test_binding_constants_match_header():
     text = open(HEADER).read()
-    vals = {k: int(v) for k, v in re.findall(r"\b(FA_TILE_[A-Z_]+)\s*=\s*(\d+)", text)}
-    assert vals == {"FA_TILE_REVERSE": fa.TILE_REVERSE, "FA_TILE_L_ROUNDED": fa.TILE_L_ROUNDED}
+    vals = {k: int(v) for k, v in re.findall(r"\b(FA_TILE_[A-Z0-9_]+)\s*=\s*(\d+)", text)}
+    assert vals == {"FA_TILE_REVERSE": fa.TILE_REVERSE, "FA_TILE_L_ROUNDED": fa.TILE_L_ROUNDED,
+                    "FA_TILE_TENSOR_CORE": fa.TILE_TENSOR_CORE, "FA_TILE_O_F32": fa.TILE_O_F32}
+    vals = {k: int(v) for k, v in re.findall(r"\b(FA_BWD_DKDV_[A-Z]+)\s*=\s*(\d+)", text)}
+    assert vals == {"FA_BWD_DKDV_PAIR": fa.BWD_DKDV_PAIR, "FA_BWD_DKDV_SINGLE": fa.BWD_DKDV_SINGLE}
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -121,9 +124,17 @@ def test_aux_entry_validation(lib):
                                      None) == INVALID
     assert lib.fa_fwd_tile_reference(A, A, A, A, A, 1, 1, 64, 192, 0.125, 0, None, None, 64, 0,
                                      None) == UNSUPPORTED
-    assert lib.fa_fwd_tile_reference(A, A, A, A, A, 1, 1, 64, 64, 0.125, 0, None, None, 64, 4,
+    assert lib.fa_fwd_tile_reference(A, A, A, A, A, 1, 1, 64, 64, 0.125, 0, None, None, 64, 16,
                                      None) == INVALID
     assert "flags" in lib.fa_get_last_error().decode()
+    # the tensor-core sweep: d = 64 and bc in {64, 128} only, no reverse / rounded-l variant
+    tc = fa.TILE_TENSOR_CORE
+    assert lib.fa_fwd_tile_reference(A, A, A, A, A, 1, 1, 64, 64, 0.125, 0, None, None, 64,
+                                     tc | fa.TILE_REVERSE, None) == INVALID
+    assert lib.fa_fwd_tile_reference(A, A, A, A, A, 1, 1, 64, 128, 0.125, 0, None, None, 64, tc,
+                                     None) == UNSUPPORTED
+    assert lib.fa_fwd_tile_reference(A, A, A, A, A, 1, 1, 64, 64, 0.125, 0, None, None, 96, tc,
+                                     None) == UNSUPPORTED
     assert lib.fa_naive_fwd(A, A, A, A, A, 1, 1, 64, 64, 0.125, 0, None, None, A, 16,
                             None) == WORKSPACE
 

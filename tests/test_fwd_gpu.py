@@ -181,3 +181,48 @@ def test_fwd_long_sequence_sampled(cuda_lib):
     o_ref, l_ref = oracle.attn_fwd_rows(x["q"], x["k"], x["v"], x["scale"], rows, True)
     compare_o(f64(o).reshape(-1, 64)[rows], o_ref)
     compare_lse(f64(lse).reshape(-1)[rows], l_ref)
+
+
+@pytest.mark.parametrize("bc", [64, 128])
+def test_tensor_core_tile_widths_and_fp32_output(cuda_lib, bc):
+    """The deviation study's tensor-core path: the tcgen05 forward at 64- and 128-key tiles
+    (d = 64, key padding), as bf16 O and as the fp32 O/l before its rounding.  Both are within
+    the bf16 tolerance of the oracle; the fp32 output rounds to the bf16 one (round to nearest
+    even); at 64-key tiles -- the library's own d = 64 forward -- the bf16 output is fa_fwd's,
+    bit for bit."""
+    x = syn.make_inputs(3, 2, 512, 64, "bf16", seed=15, kv_len=np.array([130, 512, 301], np.int32),
+                        with_grad=False)
+    g = to_gpu(x)
+    o_ref, lse_ref = oracle_fwd(x)
+    o, lse = cuda_lib.fwd_tile_reference(g["q"], g["k"], g["v"], bc, g["scale"],
+                                         kv_len=g["kv_len"], tensor_core=True)
+    o32, lse32 = cuda_lib.fwd_tile_reference(g["q"], g["k"], g["v"], bc, g["scale"],
+                                             kv_len=g["kv_len"], tensor_core=True, o_f32=True)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_status() == 0
+    assert o32.dtype == torch.float32
+    compare_o(f64(o), o_ref)
+    compare_o(f64(o32), o_ref)
+    compare_lse(f64(lse), lse_ref)
+    assert torch.equal(o32.to(torch.bfloat16), o) and torch.equal(lse32, lse)
+    # the fp32 output is closer to the oracle than its bf16 rounding, on average
+    assert np.abs(f64(o32) - o_ref).mean() < np.abs(f64(o) - o_ref).mean()
+    if bc == 64:
+        o_lib, _ = cuda_lib.fwd(g["q"], g["k"], g["v"], g["scale"], kv_len=g["kv_len"])
+        torch.cuda.synchronize()
+        assert torch.equal(o_lib, o)
+
+
+def test_tile_reference_fp32_output(cuda_lib):
+    """The CUDA-core tile reference with fp32 output: within tolerance, and its bf16 rounding is
+    the reference's own bf16 output."""
+    x = syn.make_inputs(2, 2, 520, 64, "bf16", seed=16, causal=True, with_grad=False)
+    g = to_gpu(x)
+    o_ref, _ = oracle_fwd(x)
+    for bc in (64, 256):
+        o, _ = cuda_lib.fwd_tile_reference(g["q"], g["k"], g["v"], bc, g["scale"], True)
+        o32, _ = cuda_lib.fwd_tile_reference(g["q"], g["k"], g["v"], bc, g["scale"], True,
+                                             o_f32=True)
+        torch.cuda.synchronize()
+        compare_o(f64(o32), o_ref)
+        assert torch.equal(o32.to(torch.bfloat16), o)
