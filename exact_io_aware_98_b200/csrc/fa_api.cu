@@ -125,19 +125,20 @@ int make_map(CUtensorMap* map, const void* base, int BH, int N, int d, int box_r
   return FA_OK;
 }
 
-// 3-D view [B*H][N][d] of the fp32 dQ accumulator for TMA reduce-adds: unswizzled boxes of
-// 32 columns x 64 rows.
-int make_dq_map(CUtensorMap* map, float* base, int BH, int N, int d) {
+// 3-D view [B*H][N][d] of the fp32 dQ accumulator for TMA reduce-adds: boxes of 32 columns x
+// `box_rows` rows, unswizzled (d = 128) or 128-byte swizzled (d = 64).
+int make_dq_map(CUtensorMap* map, float* base, int BH, int N, int d, int box_rows, bool swz) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                               static_cast<cuuint64_t>(BH)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4,
                                  static_cast<cuuint64_t>(N) * d * 4};
-  const cuuint32_t box[3] = {32u, 64u, 1u};
+  const cuuint32_t box[3] = {32u, static_cast<cuuint32_t>(box_rows), 1u};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "tensor map for the dQ accumulator failed (%d)", (int)r);
   return FA_OK;
@@ -231,11 +232,10 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void
   if ((rc = make_map(&mk, k, B * H_kv, N, D, 128, "k")) != FA_OK) return rc;
   if ((rc = make_map(&mv, v, B * H_kv, N, D, 128, "v")) != FA_OK) return rc;
   if ((rc = make_map(&mdo, dO, BH, N, D, L::BM, "dO")) != FA_OK) return rc;
-  if (L::V_IN_TMEM) {
-    if ((rc = make_dq_map(&mdq, reinterpret_cast<float*>(wsb + ws.dq), BH, N, D)) != FA_OK) return rc;
-  } else {
-    mdq = mq;  // not read at d = 64 (dQ by vector atomics)
-  }
+  // d = 128: [64 rows][32 d] boxes staged in the V tile; d = 64: swizzled [32 rows][32 d] boxes
+  if ((rc = make_dq_map(&mdq, reinterpret_cast<float*>(wsb + ws.dq), BH, N, D,
+                        L::V_IN_TMEM ? 64 : 32, !L::V_IN_TMEM)) != FA_OK)
+    return rc;
   if ((rc = set_smem(fa::fa_bwd_sm100_kernel<D>, L::SMEM_ALLOC)) != FA_OK) return rc;
   fa::BwdParams p;
   p.block_mask = bm;

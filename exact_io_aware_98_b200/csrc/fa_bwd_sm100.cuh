@@ -23,9 +23,11 @@
 //   dK  += dS^T Q    (M=128, N=D, K=BM)           TMEM x smem  -> TMEM
 //   D=64 : dQ   = dS K     (M=BM=128, N=64,  K=128) smem x smem -> TMEM (row per lane)
 //   D=128: dQ^T = K^T dS^T (M=128,    N=BM=64, K=128) smem x smem -> TMEM (column per lane)
-//   dQ warpgroup: TMEM -> the fp32 dQ workspace, by vector red.global.add at D=64 and at
-//   D=128 by one TMA reduce-add per warp of a [64 rows][32 d] box staged in the V tile's
-//   shared memory (free once V is in TMEM).
+//   dQ warpgroup: TMEM -> the fp32 dQ workspace by TMA reduce-adds of boxes staged in shared
+//   memory: at D=128 one per warp of a [64 rows][32 d] box in the V tile's shared memory (free
+//   once V is in TMEM); at D=64 two per warp of [32 rows][32 d] boxes (128-byte swizzled) in the
+//   dS^T buffer the step's dQ MMA has just finished reading, handed back to the compute
+//   warpgroups once the reduce-adds have read it.
 // Hand-offs per step: P ready (-> dV(t), then S(t+1)) and dS ready (-> dK(t), then dP(t+1),
 // then dQ(t)).  In-order MMA execution lets S(t+1) reuse the TMEM that dV(t) read P^T(t) from,
 // and dP(t+1) the TMEM of dS^T(t); the compute warpgroups compute dS(t) while dV(t) and S(t+1)
@@ -75,8 +77,8 @@ struct BwdLayout {
   static constexpr int OFF_DVEC = OFF_LSE + QST * BM * 4;
   static constexpr int OFF_BAR = OFF_DVEC + QST * BM * 4;
   // kv, q_full[QST], q_empty[QST], s_full, dp_full, p_full, ds_full, dq_full[2], dq_empty[2],
-  // kv_done, fin, v_tmem
-  static constexpr int NBAR = 1 + 2 * QST + 4 + 2 + 2 + 1 + 1 + 1;
+  // kv_done, fin, v_tmem, ds_free[2]
+  static constexpr int NBAR = 1 + 2 * QST + 4 + 2 + 2 + 1 + 1 + 1 + 2;
   static constexpr int THREADS = 448;
   static constexpr int HALF = BM / 2;               // query columns per compute warpgroup
   static constexpr int NCH = HALF / 32;             // 32-column chunks per compute warpgroup
@@ -102,6 +104,9 @@ struct BwdLayout {
   static_assert(!V_IN_TMEM || VT_COL + D / 2 <= DV_COL, "TMEM: V overlaps dV");
   static constexpr int DQ_STAGE = 64 * 32 * 4;         // one dQ warp's [64 rows][32 d] fp32 box
   static_assert(!V_IN_TMEM || 4 * DQ_STAGE <= KV_TILE, "dQ staging fits in the V tile");
+  // d = 64: one dQ warp's [32 rows][64 d] fp32 box, staged as two swizzled [32][32] halves
+  static constexpr int DQ64_STAGE = 32 * 64 * 4;
+  static_assert(V_IN_TMEM || 4 * DQ64_STAGE <= DS_TILE, "dQ staging fits in a dS^T buffer");
   static_assert(DK_COL + D <= TMEM_COLS, "TMEM budget");
 };
 
@@ -115,7 +120,8 @@ enum : int {
 
 template <int D>
 // 14 warps: some SM sub-partitions hold four of them, which caps registers at 128 per thread.
-// tm_dq: the fp32 dQ accumulator [B*H][N][D], boxes of 32 columns x 64 rows (d = 128 only).
+// tm_dq: the fp32 dQ accumulator [B*H][N][D], boxes of 32 columns x 64 rows (d = 128) or of
+// 32 columns x 32 rows with the 128-byte swizzle (d = 64).
 __global__ void __launch_bounds__(448, 1)
 fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -146,6 +152,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint64_t* bar_done = bar_dqe + 2;
   uint64_t* bar_fin = bar_done + 1;
   uint64_t* bar_vt = bar_fin + 1;        // V copied into TMEM (d = 128)
+  uint64_t* bar_dsf = bar_vt + 1;        // [2] d = 64: dS^T buffer free again (dQ staged out)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
   const float* s_lse = reinterpret_cast<const float*>(smem + L::OFF_LSE);
@@ -212,6 +219,8 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(bar_done, 1);
     mbar_init(bar_fin, 1);
     mbar_init(bar_vt, 128);
+    mbar_init(&bar_dsf[0], 4);
+    mbar_init(&bar_dsf[1], 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -517,7 +526,13 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_arrive(bar_p);
       // ---- dS = P (dP - Dvec): bf16 into TMEM (over my dP^T) and into smem for the dQ MMA
       got = mbar_wait(bar_dp, t & 1, abort_flag, SITE_BWD_C_DP);
-      if (t >= 2) got = got && mbar_wait(&bar_dqf[buf], ((t - 2) >> 1) & 1, abort_flag, SITE_BWD_C_DQ);
+      // dS^T buffer buf was read by dQ(t-2) and, at d = 64, then held dQ(t-2)'s staged boxes
+      if (t >= 2) {
+        if constexpr (L::V_IN_TMEM)
+          got = got && mbar_wait(&bar_dqf[buf], ((t - 2) >> 1) & 1, abort_flag, SITE_BWD_C_DQ);
+        else
+          got = got && mbar_wait(&bar_dsf[buf], ((t - 2) >> 1) & 1, abort_flag, SITE_BWD_C_DQ);
+      }
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
       uint8_t* ds_row = smem + L::OFF_DS + buf * L::DS_TILE + jl * 128;
@@ -624,17 +639,30 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       tc_fence_before();
       mbar_arrive(&bar_dqe[buf]);
       if constexpr (D == 64) {
-        // lane = query row i0 + 32qw + lane, 64 columns of dQ
-        const int qi = i0 + 32 * qw + lane;
-        if (qi < N) {
-          float4* dst = reinterpret_cast<float4*>(p.dq_acc + (static_cast<size_t>(bh) * N + qi) * D);
+        // lane = query row i0 + 32qw + lane, 64 columns of dQ: staged as this warp's [32 rows]
+        // [64 d] box in dS^T buffer buf (dQ(t), the last reader of that buffer, has completed),
+        // as two [32 rows][32 d] halves with the 128-byte swizzle (16-byte chunk c of row r at
+        // chunk c ^ (r & 7): the 32 lanes' stores spread over all banks), and added to the
+        // accumulator by two TMA reduce-adds (rows >= N are skipped).  Once the reduce-adds have
+        // read the box, the buffer goes back to the compute warpgroups.
+        uint8_t* stg = smem + L::OFF_DS + buf * L::DS_TILE + qw * L::DQ64_STAGE;
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const uint32_t* src = &v[u >> 3][(u & 7) * 4];
-            atomicAdd(dst + u, make_float4(__uint_as_float(src[0]), __uint_as_float(src[1]),
-                                           __uint_as_float(src[2]), __uint_as_float(src[3])));
-          }
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<float4*>(stg + hh * 4096 + lane * 128 + ((c ^ (lane & 7)) * 16)) =
+                make_float4(__uint_as_float(v[hh][4 * c]), __uint_as_float(v[hh][4 * c + 1]),
+                            __uint_as_float(v[hh][4 * c + 2]), __uint_as_float(v[hh][4 * c + 3]));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(&tm_dq, stg, 0, i0 + 32 * qw, bh);
+          tma_reduce_add_3d(&tm_dq, stg + 4096, 32, i0 + 32 * qw, bh);
+          bulk_commit_group();
+          bulk_wait_read_all();
+          mbar_arrive(&bar_dsf[buf]);
         }
+        __syncwarp();
       } else {
         // lane = head dimension 32qw + lane, columns = query rows i0 .. i0+63: staged as this
         // warp's [64][32] fp32 box in the V tile (V lives in TMEM by now: dQ(0) follows the
@@ -655,10 +683,8 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       ++t;
     }
-    if (L::V_IN_TMEM) {
-      if (lane == 0) bulk_wait_all();  // the reductions are complete before the CTA ends
-      __syncwarp();
-    }
+    if (lane == 0) bulk_wait_all();  // the reductions are complete before the CTA ends
+    __syncwarp();
   }
 
   tc_fence_before();
