@@ -121,8 +121,8 @@ def traffic_for(kernel: str, workload: str):
         return None
     with open(path) as f:
         t = json.load(f)
-    e = t.get(kernel, {})
-    if e.get("workload") != workload or e.get("csrc_hash") != csrc_hash():
+    e = t.get(kernel, {}).get(workload, {})
+    if e.get("csrc_hash") != csrc_hash():
         return None
     return e.get("bytes_per_launch")
 
