@@ -189,12 +189,16 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                int H_kv, int N, float scale, int causal, const uint8_t* bm,
                const int32_t* kv_len, cudaStream_t stream) {
   using L = fa::FwdLayout<D, BN>;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   const int BH = B * H;
   int rc;
   if ((rc = make_map(&mq, q, BH, N, D, 128, "q")) != FA_OK) return rc;
   if ((rc = make_map(&mk, k, B * H_kv, N, D, L::BN, "k")) != FA_OK) return rc;
   if ((rc = make_map(&mv, v, B * H_kv, N, D, L::BN, "v")) != FA_OK) return rc;
+  // bf16 O: one warp's [32 rows][64 d] boxes (the fp32 O/l of the deviation study is stored
+  // per lane, so its map is never used: it is built over o with the bf16 layout only to fill
+  // the parameter)
+  if ((rc = make_map(&mo, o, BH, N, D, 32, "o")) != FA_OK) return rc;
   if ((rc = set_smem(fa::fa_fwd_sm100_kernel<D, BN, O32>, L::SMEM_ALLOC)) != FA_OK) return rc;
   fa::FwdParams p;
   p.block_mask = bm;
@@ -216,7 +220,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   const long long grid = static_cast<long long>(p.n_mtiles) * BH;
   if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
   TimedLaunch tl("fa_fwd_sm100_kernel", stream);
-  fa::fa_fwd_sm100_kernel<D, BN, O32><<<static_cast<unsigned>(grid), 320, L::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
+  fa::fa_fwd_sm100_kernel<D, BN, O32><<<static_cast<unsigned>(grid), 320, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mo, p);
   return check_launch("fa_fwd_sm100_kernel");
 }
 
@@ -225,13 +229,16 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void
                int B, int H, int H_kv, int N, float scale, int causal, const uint8_t* bm,
                const int32_t* kv_len, const BwdWs& ws, uint8_t* wsb, cudaStream_t stream) {
   using L = fa::BwdLayout<D>;
-  CUtensorMap mq, mk, mv, mdo, mdq;
+  CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv;
   const int BH = B * H;
   int rc;
   if ((rc = make_map(&mq, q, BH, N, D, L::BM, "q")) != FA_OK) return rc;
   if ((rc = make_map(&mk, k, B * H_kv, N, D, 128, "k")) != FA_OK) return rc;
   if ((rc = make_map(&mv, v, B * H_kv, N, D, 128, "v")) != FA_OK) return rc;
   if ((rc = make_map(&mdo, dO, BH, N, D, L::BM, "dO")) != FA_OK) return rc;
+  // dK, dV: one warp's [32 rows][64 d] boxes
+  if ((rc = make_map(&mdk, dk, B * H_kv, N, D, 32, "dK")) != FA_OK) return rc;
+  if ((rc = make_map(&mdv, dv, B * H_kv, N, D, 32, "dV")) != FA_OK) return rc;
   // d = 128: [64 rows][32 d] boxes staged in the V tile; d = 64: swizzled [32 rows][32 d] boxes
   if ((rc = make_dq_map(&mdq, reinterpret_cast<float*>(wsb + ws.dq), BH, N, D,
                         L::V_IN_TMEM ? 64 : 32, !L::V_IN_TMEM)) != FA_OK)
@@ -264,7 +271,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void
   const long long grid = static_cast<long long>(p.n_ktiles) * B * H_kv;  // one CTA per K/V tile
   if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
   TimedLaunch tl("fa_bwd_sm100_kernel", stream);
-  fa::fa_bwd_sm100_kernel<D><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, mdq, p);
+  fa::fa_bwd_sm100_kernel<D><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, mdq, mdk, mdv, p);
   return check_launch("fa_bwd_sm100_kernel");
 }
 
@@ -275,13 +282,15 @@ int launch_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
                     const uint8_t* bm, const int32_t* kv_len, const BwdWs& ws, uint8_t* wsb,
                     cudaStream_t stream) {
   using L = fa::BwdDkdvLayout<D>;
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv;
   const int BH = B * H;
   int rc;
   if ((rc = make_map(&mq, q, BH, N, D, L::BM, "q")) != FA_OK) return rc;
   if ((rc = make_map(&mk, k, B * H_kv, N, D, 128, "k")) != FA_OK) return rc;
   if ((rc = make_map(&mv, v, B * H_kv, N, D, 128, "v")) != FA_OK) return rc;
   if ((rc = make_map(&mdo, dO, BH, N, D, L::BM, "dO")) != FA_OK) return rc;
+  if ((rc = make_map(&mdk, dk, B * H_kv, N, D, 32, "dK")) != FA_OK) return rc;  // [32][64] boxes
+  if ((rc = make_map(&mdv, dv, B * H_kv, N, D, 32, "dV")) != FA_OK) return rc;
   if ((rc = set_smem(fa::fa_bwd_dkdv_sm100_kernel<D>, L::SMEM_ALLOC)) != FA_OK) return rc;
   fa::BwdParams p;
   p.block_mask = bm;
@@ -310,7 +319,7 @@ int launch_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
   const long long grid = static_cast<long long>(p.n_ktiles) * B * H_kv;
   if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
   TimedLaunch tl("fa_bwd_dkdv_sm100_kernel", stream);
-  fa::fa_bwd_dkdv_sm100_kernel<D><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, p);
+  fa::fa_bwd_dkdv_sm100_kernel<D><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
   return check_launch("fa_bwd_dkdv_sm100_kernel");
 }
 

@@ -83,7 +83,9 @@ __global__ void __launch_bounds__(320, 1)
 fa_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v,
-                         const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+                         const __grid_constant__ CUtensorMap tm_do,
+                         const __grid_constant__ CUtensorMap tm_dk,
+                         const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
   using L = BwdDkdvLayout<D>;
   constexpr int BM = L::BM;
   extern __shared__ uint8_t smem_raw[];
@@ -406,9 +408,14 @@ fa_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       tc_fence_after();
     }
     if (ok) {
+      // This warp's 32 key rows are staged as D/64 [32 rows][64 d] bf16 boxes with the 128-byte
+      // swizzle (16-byte chunk c of row r at chunk c ^ (r & 7)) in the Q ring, which no MMA or
+      // load touches any more (bar_done follows the last MMA), and written by one TMA store per
+      // box (rows past N are not written) instead of one memory transaction per lane and store.
       const uint32_t col0 = h == 0 ? L::DV_COL : L::DK_COL;
       const float mul = h == 0 ? 1.0f : p.scale;
-      __nv_bfloat16* dst_row = (h == 0 ? p.dv : p.dk) + (static_cast<size_t>(bhk) * N + kj) * D;
+      uint8_t* stg = smem + L::OFF_Q + warp * (D / 64) * 4096;
+      static_assert(8 * (D / 64) * 4096 <= L::QST * L::Q_TILE, "dK/dV staging fits the Q ring");
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t gr[32];
@@ -424,13 +431,24 @@ fa_bwd_dkdv_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           hv[i] = pack_bf16x2(__uint_as_float(gr[2 * i]) * mul, __uint_as_float(gr[2 * i + 1]) * mul);
-        if (kj < N) {
-          uint4* dst = reinterpret_cast<uint4*>(dst_row + 32 * c);
+        uint8_t* box = stg + (c >> 1) * 4096 + lane * 128;
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+        for (int i = 0; i < 4; ++i) {
+          const int q = (c & 1) * 4 + i;  // 16-byte chunk of the 128-byte row
+          *reinterpret_cast<uint4*>(box + ((q ^ (lane & 7)) * 16)) =
+              make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
         }
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < D / 64; ++s)
+          tma_store_3d(h == 0 ? &tm_dv : &tm_dk, stg + s * 4096, 64 * s, k0 + 32 * qw, bhk);
+        bulk_commit_group();
+        bulk_wait_read_all();  // the boxes have been read before the CTA ends
+      }
+      __syncwarp();
     }
   }
 

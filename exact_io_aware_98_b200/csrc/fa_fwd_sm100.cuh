@@ -110,7 +110,8 @@ template <int D, int BN_ = fwd_bn<D>(), bool O32 = false>
 __global__ void __launch_bounds__(320, FwdLayout<D, BN_>::CTAS_PER_SM)
 fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_o, const FwdParams p) {
   using L = FwdLayout<D, BN_>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -474,9 +475,23 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         ok = __all_sync(0xffffffffu, got);
         tc_fence_after();
       }
+      // bf16 O at d = 64: this warp's 32 rows staged as a [32 rows][64 d] box with the 128-byte
+      // swizzle (16-byte chunk c of row r at chunk c ^ (r & 7)) in its own Q tile, which no MMA
+      // reads any more (the last P.V of this Q tile has finished, and every S MMA before it), then
+      // one TMA store (rows past N are not written).  Per-lane 16-byte stores to rows 2D bytes
+      // apart cost one memory transaction per lane, which two CTAs per SM feel in every CTA's
+      // turnaround; at d = 128 (one CTA per SM) those stores drain after the CTA has gone,
+      // while the TMA store's read of the staging box would sit on the CTA's exit.
+      constexpr bool TMA_O = !O32 && D == 64;
+      if constexpr (TMA_O) {
+        // no key tile for this Q tile (no keys, or its block-mask row is empty): the Q load the
+        // staging area belongs to may still be in flight
+        if (cnt == 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, abort_flag, SITE_FWD_SM_O));
+      }
       const float inv = (l > 0.f) ? 1.0f / l : 0.0f;
-      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * N + row) * D;
       float* orow32 = p.o32 + (static_cast<size_t>(bh) * N + row) * D;
+      uint8_t* stg = smem + L::OFF_Q + w * L::TILE + qw * (D / 64) * 4096;
+      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * N + row) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -501,13 +516,34 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             h[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-          if (row < N) {
+          if constexpr (TMA_O) {
+            uint8_t* box = stg + (c >> 1) * 4096 + lane * 128;
+            if (ok) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int q = (c & 1) * 4 + i;  // 16-byte chunk of the 128-byte row
+                *reinterpret_cast<uint4*>(box + ((q ^ (lane & 7)) * 16)) =
+                    make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+              }
+            }
+          } else if (row < N) {
             uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
               dst[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
           }
         }
+      }
+      if (TMA_O && ok) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+          for (int s = 0; s < D / 64; ++s) tma_store_3d(&tm_o, stg + s * 4096, 64 * s, q0 + 32 * qw, bh);
+          bulk_commit_group();
+          bulk_wait_read_all();  // the boxes have been read before the CTA ends
+        }
+        __syncwarp();
       }
       if (row < N)
         p.lse[static_cast<size_t>(bh) * N + row] =
