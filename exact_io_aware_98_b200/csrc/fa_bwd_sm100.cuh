@@ -77,8 +77,8 @@ struct BwdLayout {
   static constexpr int OFF_DVEC = OFF_LSE + QST * BM * 4;
   static constexpr int OFF_BAR = OFF_DVEC + QST * BM * 4;
   // kv, q_full[QST], q_empty[QST], s_full, dp_full, p_full, ds_full, dq_full[2], dq_empty[2],
-  // kv_done, fin, v_tmem, ds_free[2]
-  static constexpr int NBAR = 1 + 2 * QST + 4 + 2 + 2 + 1 + 1 + 1 + 2;
+  // kv_done, fin, v_tmem, ds_free[2], dv_done
+  static constexpr int NBAR = 1 + 2 * QST + 4 + 2 + 2 + 1 + 1 + 1 + 2 + 1;
   static constexpr int THREADS = 448;
   static constexpr int HALF = BM / 2;               // query columns per compute warpgroup
   static constexpr int NCH = HALF / 32;             // 32-column chunks per compute warpgroup
@@ -94,6 +94,10 @@ struct BwdLayout {
   // then stages dQ^T for TMA reduce-adds into the fp32 accumulator (no per-element atomics).
   // The 64 TMEM columns come from holding one dQ^T buffer instead of two.
   static constexpr bool V_IN_TMEM = D == 128;
+  // d = 64: warpgroup 0 writes dV as soon as the last dV MMA has finished (before the last dK
+  // and dQ MMAs), staging it in the dS^T buffer the last two steps no longer use.  At d = 128 a
+  // dS^T buffer (16 KB) cannot hold dV (32 KB).
+  static constexpr bool EARLY_DV = !V_IN_TMEM;
   static constexpr int DQB = V_IN_TMEM ? 1 : 2;         // dQ buffers of 64 columns
   static constexpr uint32_t S_COL = 0;
   static constexpr uint32_t DP_COL = BM;
@@ -155,6 +159,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint64_t* bar_fin = bar_done + 1;
   uint64_t* bar_vt = bar_fin + 1;        // V copied into TMEM (d = 128)
   uint64_t* bar_dsf = bar_vt + 1;        // [2] d = 64: dS^T buffer free again (dQ staged out)
+  uint64_t* bar_dvd = bar_dsf + 2;       // EARLY_DV: the last dV MMA has finished
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
   const float* s_lse = reinterpret_cast<const float*>(smem + L::OFF_LSE);
@@ -223,6 +228,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(bar_vt, 128);
     mbar_init(&bar_dsf[0], 4);
     mbar_init(&bar_dsf[1], 4);
+    mbar_init(bar_dvd, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -386,6 +392,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!mbar_wait_w(bar_p, t & 1, abort_flag, SITE_BWD_MMA_P)) { ok = false; break; }
         tc_fence_after();
         mma_grad(L::S_COL, do_mn, st, L::DV_COL, t > 0);
+        if (L::EARLY_DV && !next) mma_commit_w(bar_dvd);
         if (next) {
           if (!mbar_wait_w(&bar_qf[st1], ((t + 1) / L::QST) & 1, abort_flag, SITE_BWD_MMA_Q)) {
             ok = false;
@@ -585,8 +592,13 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     // ---------------------------------------------------------------- epilogue: dK, dV
     // warpgroup 0 writes dV, warpgroup 1 writes dK (x scale)
+    const bool early = L::EARLY_DV && h == 0 && n_steps > 0;
     if (ok && n_steps > 0) {
-      const bool got = mbar_wait(bar_done, 0, abort_flag, SITE_BWD_C_DONE);
+      // early dV: its staging buffer held dS(t-2), last read by dQ(t-2) (finished before the
+      // last dV) and by the dQ warps' boxes of that step
+      bool got = mbar_wait(early ? bar_dvd : bar_done, 0, abort_flag, SITE_BWD_C_DONE);
+      if (early && t >= 2)
+        got = got && mbar_wait(&bar_dsf[t & 1], ((t - 2) >> 1) & 1, abort_flag, SITE_BWD_C_DQ);
       ok = __all_sync(0xffffffffu, got);
       tc_fence_after();
     }
@@ -598,8 +610,10 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       // Per-lane 16-byte stores to rows 2D bytes apart cost one memory transaction per lane.
       const uint32_t col0 = h == 0 ? L::DV_COL : L::DK_COL;
       const float mul = h == 0 ? 1.0f : p.scale;
-      uint8_t* stg = smem + L::OFF_Q + warp * (D / 64) * 4096;
+      uint8_t* stg = early ? smem + L::OFF_DS + (t & 1) * L::DS_TILE + warp * (D / 64) * 4096
+                           : smem + L::OFF_Q + warp * (D / 64) * 4096;
       static_assert(8 * (D / 64) * 4096 <= L::QST * L::Q_TILE, "dK/dV staging fits the Q ring");
+      static_assert(!L::EARLY_DV || 4 * (D / 64) * 4096 <= L::DS_TILE, "dV staging fits a dS^T buffer");
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t g[32];
