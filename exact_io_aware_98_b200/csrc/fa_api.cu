@@ -183,8 +183,9 @@ BwdWs bwd_ws(int B, int H, int N, int d) {
   return w;
 }
 
-// BN: keys per KV tile; O32: o is fp32 O/l (deviation study) instead of bf16 O.
-template <int D, int BN = fa::fwd_bn<D>(), bool O32 = false>
+// BN: keys per KV tile; O32: o is fp32 O/l (deviation study) instead of bf16 O; RANKED: the
+// CTAs order the Q tiles by their unmasked blocks (needs a block mask and N <= 16384).
+template <int D, int BN = fa::fwd_bn<D>(), bool O32 = false, bool RANKED = false>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                int H_kv, int N, float scale, int causal, const uint8_t* bm,
                const int32_t* kv_len, cudaStream_t stream) {
@@ -199,7 +200,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   // per lane, so its map is never used: it is built over o with the bf16 layout only to fill
   // the parameter)
   if ((rc = make_map(&mo, o, BH, N, D, 32, "o")) != FA_OK) return rc;
-  if ((rc = set_smem(fa::fa_fwd_sm100_kernel<D, BN, O32>, L::SMEM_ALLOC)) != FA_OK) return rc;
+  if ((rc = set_smem(fa::fa_fwd_sm100_kernel<D, BN, O32, RANKED>, L::SMEM_ALLOC)) != FA_OK) return rc;
   fa::FwdParams p;
   p.block_mask = bm;
   p.kv_len = kv_len;
@@ -220,7 +221,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   const long long grid = static_cast<long long>(p.n_mtiles) * BH;
   if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
   TimedLaunch tl("fa_fwd_sm100_kernel", stream);
-  fa::fa_fwd_sm100_kernel<D, BN, O32><<<static_cast<unsigned>(grid), 320, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mo, p);
+  fa::fa_fwd_sm100_kernel<D, BN, O32, RANKED><<<static_cast<unsigned>(grid), 320, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mo, p);
   return check_launch("fa_fwd_sm100_kernel");
 }
 
@@ -449,8 +450,13 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   if ((rc = check_groups(H, H_kv)) != FA_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == FA_BF16) {
-    if (d == 64)
+    if (d == 64) {
+      // block masks: the Q tiles are taken heaviest first (a block-sparse mask need not make
+      // the last rows the longest, as a causal one does)
+      if (block_mask != nullptr && (N + 255) / 256 <= fa::FWD_RANK_TILES)
+        return launch_fwd<64, 64, false, true>(q, k, v, o, lse, B, H, H_kv, N, scale, causal, block_mask, kv_len, s);
       return launch_fwd<64>(q, k, v, o, lse, B, H, H_kv, N, scale, causal, block_mask, kv_len, s);
+    }
     if (d == 128)
       return launch_fwd<128>(q, k, v, o, lse, B, H, H_kv, N, scale, causal, block_mask, kv_len, s);
     return fail(FA_ERR_UNSUPPORTED, "bf16 forward supports d in {64, 128}, got %d", d);

@@ -86,7 +86,9 @@ struct FwdLayout {
   // p2_full[2], fin
   static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 6 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int BYTES = OFF_MISC + 16;
+  // block-mask CTA order (d = 64): per Q tile its unmasked blocks, then the Q tiles by that count
+  static constexpr int OFF_ORD = OFF_MISC + 16;
+  static constexpr int BYTES = OFF_ORD + 2 * 64 * 4;          // 2 x FWD_RANK_TILES ints
   static constexpr int SMEM_ALLOC = BYTES + 1024;   // slack for 1024-byte alignment
   static_assert(CTAS_PER_SM * (SMEM_ALLOC + 1024) <= 233472, "shared memory per SM");
   static constexpr uint32_t TMEM_COLS = 2 * BN + 2 * D <= 256 ? 256 : 512;
@@ -97,6 +99,35 @@ struct FwdLayout {
   __device__ static constexpr uint32_t s_col(int w) { return static_cast<uint32_t>(w) * BN; }
 };
 
+// Block-mask CTA order: the Q tile (256 rows) of rank `rank` when the Q tiles are ordered by
+// their number of unmasked 128 x 128 blocks (causal: on or below the diagonal), most first, ties
+// to the later Q tile.  Every thread of the CTA calls it (three barriers); s_wt and s_ord are
+// FWD_RANK_TILES ints each of shared memory.
+constexpr int FWD_RANK_TILES = 64;  // Q tiles ranked (N <= 16384)
+__device__ __noinline__ int fwd_ranked_qtile(const uint8_t* __restrict__ block_mask, int N,
+                                             int n_mtiles, int causal, int rank, int* s_wt,
+                                             int* s_ord) {
+  if (static_cast<int>(threadIdx.x) < n_mtiles) s_wt[threadIdx.x] = 0;
+  __syncthreads();
+  const int nbm = (N + 127) / 128;
+  for (int e = threadIdx.x; e < nbm * nbm; e += blockDim.x) {
+    const int r = e / nbm, c = e - r * nbm;  // query block r, key block c
+    if (block_mask[e] && (!causal || c <= r)) atomicAdd(&s_wt[r >> 1], 1);
+  }
+  __syncthreads();
+  if (static_cast<int>(threadIdx.x) < n_mtiles) {
+    const int i = threadIdx.x, wi = s_wt[i];
+    int rk = 0;
+    for (int j = 0; j < n_mtiles; ++j) {
+      const int wj = s_wt[j];
+      rk += (wj > wi || (wj == wi && j > i)) ? 1 : 0;
+    }
+    s_ord[rk] = i;
+  }
+  __syncthreads();
+  return s_ord[rank];
+}
+
 // Wait-site codes recorded in the status word on a timeout.
 enum : int {
   SITE_FWD_LOAD_EMPTY = 1, SITE_FWD_LOAD_DRAIN = 2, SITE_FWD_MMA_Q = 3, SITE_FWD_MMA_K = 4,
@@ -106,7 +137,9 @@ enum : int {
 
 // O32: write the fp32 O/l to p.o32 instead of bf16 O to p.o (the deviation study's view of the
 // output before its bf16 rounding).
-template <int D, int BN_ = fwd_bn<D>(), bool O32 = false>
+// RANKED: the CTA order ranks the Q tiles by their unmasked blocks (block-masked calls; a
+// separate instantiation, since the ranking changes the register allocation of the loop).
+template <int D, int BN_ = fwd_bn<D>(), bool O32 = false, bool RANKED = false>
 __global__ void __launch_bounds__(320, FwdLayout<D, BN_>::CTAS_PER_SM)
 fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -134,13 +167,18 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int lane = threadIdx.x & 31;
   const int BH = p.B * p.H;
   // CTA order: groups of p.hgroup heads in turn (a group's Q, K, V and O fit in L2), and
-  // inside a group the heaviest Q tiles (the last rows under a causal mask) first.
+  // inside a group the heaviest Q tiles first: the last rows under a causal mask, or, RANKED
+  // (block masks), the Q tiles with the most unmasked blocks, counted by every CTA from the
+  // mask, so that the longest CTAs do not start last.
   const int per_group = p.hgroup * p.n_mtiles;
   const int grp = static_cast<int>(blockIdx.x) / per_group;
   const int g0 = grp * p.hgroup;
   const int gn = min(p.hgroup, BH - g0);               // heads in this group (the last may have fewer)
   const int slot = static_cast<int>(blockIdx.x) - grp * per_group;
-  const int mt = p.n_mtiles - 1 - slot / gn;
+  const int mt = RANKED ? fwd_ranked_qtile(p.block_mask, p.N, p.n_mtiles, p.causal, slot / gn,
+                                           reinterpret_cast<int*>(smem + L::OFF_ORD),
+                                           reinterpret_cast<int*>(smem + L::OFF_ORD) + FWD_RANK_TILES)
+                        : p.n_mtiles - 1 - slot / gn;
   const int bh = g0 + slot % gn;
   const int b = bh / p.H;
   const int bh_kv = b * p.H_kv + (bh % p.H) / (p.H / p.H_kv);  // K/V head of this query head
