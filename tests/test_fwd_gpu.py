@@ -58,6 +58,26 @@ def test_fwd_small_elementwise(cuda_lib, case):
     compare_lse(f64(lse), lse_ref)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_random_block_masks(cuda_lib, causal):
+    """Block masks whose rows hold very different numbers of blocks (and equal ones), so that
+    the d = 64 forward's CTAs, which order the 256-row query tiles by their unmasked blocks,
+    take them in a scrambled order; with key padding in one batch entry."""
+    N = 2000
+    nb = (N + 127) // 128
+    rng = np.random.default_rng(31 + int(causal))
+    density = rng.permutation(np.linspace(0.05, 1.0, nb))  # per query block, shuffled
+    bm = (rng.random((nb, nb)) < density[:, None]).astype(np.uint8)
+    bm[3, :] = bm[4, :]                                      # equal rows
+    bm[nb - 1, :] = 0                                        # a query block with no key block
+    x = syn.make_inputs(2, 2, N, 64, "bf16", seed=90 + int(causal), causal=causal,
+                        kv_len=np.array([N, 1111], np.int32), block_mask=bm, with_grad=False)
+    o, lse = run_fwd(cuda_lib, to_gpu(x))
+    o_ref, lse_ref = oracle_fwd(x)
+    compare_o(f64(o), o_ref)
+    compare_lse(f64(lse), lse_ref)
+
+
 def test_fwd_fully_masked_rows(cuda_lib):
     """Query block 1 keeps no key block: its rows give O = 0 and lse = -inf."""
     N = 384
