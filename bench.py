@@ -198,8 +198,9 @@ def max_over_ranks(values, dist, device) -> list:
     return [float(v) for v in t.tolist()]
 
 
-# MUFU (special-function unit) throughput for ex2: 16 results per clock per SM, the nominal
-# figure for recent NVIDIA architectures; 148 SMs on a B200.
+# MUFU (special-function unit) throughput for ex2: 16 results per clock per SM, measured on a
+# B200 with independent ex2.approx chains on every SM (the packed f16x2 form gives the same 16);
+# 148 SMs on a B200.
 MUFU_PER_CLK_PER_SM = 16
 N_SM = 148
 
