@@ -48,7 +48,7 @@ typedef enum { FA_BF16 = 0, FA_F32 = 1 } fa_dtype;
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID = -1,     /* null pointer, non-positive size, bad scale, unknown dtype   */
-  FA_ERR_UNSUPPORTED = -2, /* head dimension or dtype this build has no kernel for        */
+  FA_ERR_UNSUPPORTED = -2, /* head dimension or dtype the library has no kernel for       */
   FA_ERR_ALIGN = -3,       /* a tensor pointer is not 16-byte aligned (TMA requirement)   */
   FA_ERR_CUDA = -4,        /* a CUDA call or kernel launch failed                         */
   FA_ERR_TIMEOUT = -5,     /* a device-side bounded wait gave up (see fa_device_status)  */
