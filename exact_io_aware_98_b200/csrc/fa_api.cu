@@ -10,6 +10,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "fa.h"
@@ -42,6 +43,27 @@ int check_launch(const char* what) {
   if (e != cudaSuccess) return fail(FA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FA_OK;
+}
+
+// overlap: launch with programmatic stream serialisation.  The kernel's CTAs may then start
+// while the kernel before it on the stream finishes (once each of that kernel's CTAs has started
+// and executed griddepcontrol.launch_dependents, or exited); the kernel executes
+// griddepcontrol.wait before it reads or writes anything that kernel touches.  Otherwise a plain
+// launch.
+template <typename... Exp, typename... Act>
+cudaError_t launch_ex(bool overlap, void (*kern)(Exp...), unsigned grid, unsigned block,
+                      size_t smem, cudaStream_t s, Act&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = overlap ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Act>(args)...);
 }
 
 // ---- optional per-kernel timing (fa_kernel_timing): two events around each tensor-core launch
@@ -272,7 +294,10 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dO, void
   const long long grid = static_cast<long long>(p.n_ktiles) * B * H_kv;  // one CTA per K/V tile
   if (grid > 0x7fffffffll) return fail(FA_ERR_UNSUPPORTED, "grid too large");
   TimedLaunch tl("fa_bwd_sm100_kernel", stream);
-  fa::fa_bwd_sm100_kernel<D><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(mq, mk, mv, mdo, mdq, mdk, mdv, p);
+  const cudaError_t le =
+      launch_ex(L::OVERLAP_PREV, fa::fa_bwd_sm100_kernel<D>, static_cast<unsigned>(grid),
+                L::THREADS, L::SMEM_ALLOC, stream, mq, mk, mv, mdo, mdq, mdk, mdv, p);
+  if (le != cudaSuccess) return fail(FA_ERR_CUDA, "fa_bwd_sm100_kernel: %s", cudaGetErrorString(le));
   return check_launch("fa_bwd_sm100_kernel");
 }
 
@@ -564,8 +589,12 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     rc = launch_bwd<128>(q, k, v, dO, dk, dv, B, H, H_kv, N, scale, causal, block_mask, kv_len, ws, wsb, s);
   if (rc != FA_OK) return rc;
   const long long n = static_cast<long long>(BH) * N * d;
-  fa::dq_convert_kernel<<<static_cast<unsigned>((n / 8 + 255) / 256 + 1), 256, 0, s>>>(
+  // overlapping the main kernel where that kernel overlaps the preprocess
+  const cudaError_t le = launch_ex(
+      d == 64 ? fa::BwdLayout<64>::OVERLAP_PREV : fa::BwdLayout<128>::OVERLAP_PREV,
+      fa::dq_convert_kernel, static_cast<unsigned>((n / 8 + 255) / 256 + 1), 256, 0, s,
       reinterpret_cast<const float*>(wsb + ws.dq), static_cast<__nv_bfloat16*>(dq), n, scale);
+  if (le != cudaSuccess) return fail(FA_ERR_CUDA, "dq_convert_kernel: %s", cudaGetErrorString(le));
   return check_launch("dq_convert_kernel");
 }
 

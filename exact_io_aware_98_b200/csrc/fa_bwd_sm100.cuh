@@ -98,6 +98,10 @@ struct BwdLayout {
   // and dQ MMAs), staging it in the dS^T buffer the last two steps no longer use.  At d = 128 a
   // dS^T buffer (16 KB) cannot hold dV (32 KB).
   static constexpr bool EARLY_DV = !V_IN_TMEM;
+  // d = 64: launched to overlap the preprocess kernel (programmatic dependent launch).  Its calls
+  // are short, so the launch gaps and the set-up are a visible share of them; at d = 128 they are
+  // not, and the kernel keeps a plain launch.
+  static constexpr bool OVERLAP_PREV = D == 64;
   static constexpr int DQB = V_IN_TMEM ? 1 : 2;         // dQ buffers of 64 columns
   static constexpr uint32_t S_COL = 0;
   static constexpr uint32_t DP_COL = BM;
@@ -236,6 +240,10 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     tmem_alloc(tmem_slot, L::TMEM_COLS);
     tmem_relinquish();
   }
+  // OVERLAP_PREV: set-up, the K/V loads and the first Q/dO loads run under the preprocess
+  // kernel's tail; lse2, Dvec and the zeroed dQ accumulator are touched only after grid_dep_wait.
+  // The dQ convert after this kernel may launch now.
+  if constexpr (L::OVERLAP_PREV) grid_dep_launch();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -272,6 +280,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                       s * 64, i0, bh);
         }
         const size_t off = static_cast<size_t>(bh) * p.N_pad + i0;
+        if (L::OVERLAP_PREV && t == 0) grid_dep_wait();  // lse2 and Dvec: preprocess kernel
         bulk_load(smem + L::OFF_LSE + st * BM * 4, p.lse2 + off, BM * 4, &bar_qf[st]);
         bulk_load(smem + L::OFF_DVEC + st * BM * 4, p.dvec + off, BM * 4, &bar_qf[st]);
         ++t;
@@ -650,6 +659,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else {
     // ------------------------------------------------------------------ dQ warpgroup
+    if constexpr (L::OVERLAP_PREV) grid_dep_wait();  // the preprocess zeroes the accumulator
     const int qw = warp & 3;
     const uint32_t t_lane = static_cast<uint32_t>(32 * qw) << 16;
     int t = 0;

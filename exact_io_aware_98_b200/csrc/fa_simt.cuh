@@ -241,6 +241,7 @@ bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* 
                       float* __restrict__ dvec, float* __restrict__ dq_acc, int BH, int N,
                       int N_pad) {
   constexpr int T = D / 8;  // threads per row
+  grid_dep_launch();          // the main backward kernel may start its set-up now
   const long long r = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) / T;
   const int part = threadIdx.x % T;
   if (r >= static_cast<long long>(BH) * N_pad) return;  // whole row groups leave together
@@ -283,6 +284,7 @@ bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* 
 __global__ void __launch_bounds__(256)
 dq_convert_kernel(const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dq, long long n,
                   float scale) {
+  grid_dep_wait();  // may be launched to overlap the kernel that completes the accumulator
   const long long e = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) * 8;
   if (e + 8 <= n) {
     const float4 a = *reinterpret_cast<const float4*>(dq_acc + e);

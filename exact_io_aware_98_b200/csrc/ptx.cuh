@@ -172,6 +172,13 @@ __device__ __forceinline__ void bulk_wait_read_all() {
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
+// Programmatic dependent launch.  grid_dep_wait: wait until the kernel this one was launched
+// after has completed and its writes are visible (a no-op when the launch did not ask for the
+// overlap).  grid_dep_launch: this CTA lets the kernel launched after this one start.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 // Makes this thread's generic-proxy shared-memory writes visible to the async proxy
 // (tcgen05.mma operand reads, TMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
