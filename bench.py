@@ -565,8 +565,8 @@ def deviation_sweep():
 def workload_measurement(name: str, iters: int = 20, flush_bytes: int = 256 << 20) -> dict:
     """fa_fwd and fa_bwd on one of the other workloads: CUDA events per call, then, in a second
     pass, each tensor-core kernel's own launches (events the library records around them; those
-    events sit between the backward's launches and stop them overlapping, so the calls are timed
-    without them).  These inputs fit in L2, so a buffer larger than L2 is overwritten before
+    events are recorded between the backward's launches and can stop them overlapping, so the
+    calls are timed without them).  These inputs fit in L2, so a buffer larger than L2 is overwritten before
     every step."""
     import exact_io_aware_98_b200 as fa
     w = syn.WORKLOADS[name]
